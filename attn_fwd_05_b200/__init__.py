@@ -1,0 +1,20 @@
+"""Exact attention for one NVIDIA B200 (sm_100a) behind a small C ABI.
+
+The CUDA library (``libattn_b200.so``, built from ``csrc/``) does all the
+work; this package only marshals torch tensors into its entry points.  The
+library is loaded on first use and a missing or unloadable library raises
+``RuntimeError``: there is no CPU fallback.
+"""
+
+from .binding import (  # noqa: F401
+    AttnError,
+    attn_decode_paged,
+    attn_decode_paged_workspace_size,
+    attn_fwd,
+    attn_fwd_ex,
+    attn_get_device_status,
+    attn_debug_watchdog,
+    attn_status_string,
+    library_path,
+    load_library,
+)

@@ -1,0 +1,166 @@
+"""ctypes binding of libattn_b200.so: argument marshalling only.
+
+Each function here has the name of a C entry point of include/attn_b200.h.  It checks
+that torch tensors have the dtype, device and layout the C side expects, reads their
+sizes and device addresses, and calls the C function on the given (default: current)
+CUDA stream.  All computation happens in the library's kernels.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+_LOCK = threading.Lock()
+
+ATTN_OK = 0
+STATUS_NAMES = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_ALIGNMENT",
+                4: "ATTN_ERR_CUDA", 5: "ATTN_ERR_DEVICE_TIMEOUT", 6: "ATTN_ERR_BAD_PAGE",
+                7: "ATTN_ERR_WORKSPACE"}
+DTYPE_BF16, DTYPE_F32 = 0, 1
+
+# exported symbol -> (restype, argtypes); mirrors include/attn_b200.h
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+SIGNATURES = {
+    "attn_abi_version": (_I, []),
+    "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P]),
+    "attn_fwd_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P]),
+    "attn_decode_paged_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
+    "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P,
+                               ctypes.c_size_t, _P]),
+    "attn_debug_watchdog": (_I, [ctypes.c_uint64, _P]),
+    "attn_get_device_status": (_I, [_P]),
+    "attn_status_string": (ctypes.c_char_p, [_I]),
+}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libattn_b200.so")
+
+
+def load_library() -> ctypes.CDLL:
+    """Loads the CUDA library; raises RuntimeError if it is missing or cannot be loaded."""
+    global _LIB
+    with _LOCK:
+        if _LIB is None:
+            path = library_path()
+            if not os.path.exists(path):
+                raise RuntimeError(f"{path} is not built: run `python -m attn_fwd_05_b200.build`")
+            lib = ctypes.CDLL(path)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _LIB = lib
+    return _LIB
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(status: int, where: str) -> None:
+    if status != ATTN_OK:
+        raise AttnError(status, where)
+
+
+def _dev(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int | None = None) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got {t.dim()}")
+    return t.data_ptr()
+
+
+def attn_fwd_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor | None,
+                causal: bool, scale: float, stream=None) -> None:
+    """Prefill forward; o is bf16 or fp32 [B, Hq, Nq, d], lse fp32 [B, Hq, Nq] or None."""
+    lib = load_library()
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if tuple(k.shape) != (B, Hkv, Nk, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k and v must be [B, Hkv, Nk, d] with q's B and d")
+    if tuple(o.shape) != (B, Hq, Nq, d):
+        raise ValueError("o must be [B, Hq, Nq, d]")
+    if lse is not None and tuple(lse.shape) != (B, Hq, Nq):
+        raise ValueError("lse must be [B, Hq, Nq]")
+    if o.dtype == torch.bfloat16:
+        odt = DTYPE_BF16
+    elif o.dtype == torch.float32:
+        odt = DTYPE_F32
+    else:
+        raise TypeError("o must be bf16 or fp32")
+    st = lib.attn_fwd_ex(_dev(q, "q", torch.bfloat16, 4), _dev(k, "k", torch.bfloat16, 4),
+                         _dev(v, "v", torch.bfloat16, 4), _dev(o, "o", o.dtype, 4), odt,
+                         None if lse is None else _dev(lse, "lse", torch.float32, 3),
+                         B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), _stream(stream))
+    _check(st, "attn_fwd_ex")
+
+
+def attn_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
+    """Prefill forward with bf16 output (see attn_fwd_ex)."""
+    if o.dtype != torch.bfloat16:
+        raise TypeError("attn_fwd writes bf16 o; use attn_fwd_ex for fp32")
+    attn_fwd_ex(q, k, v, o, lse, causal, scale, stream)
+
+
+def attn_decode_paged_workspace_size(num_seqs: int, Hq: int, Hkv: int, d: int, max_pages_per_seq: int,
+                                     page_size: int) -> int:
+    return int(load_library().attn_decode_paged_workspace_size(num_seqs, Hq, Hkv, d, max_pages_per_seq,
+                                                               page_size))
+
+
+def attn_decode_paged(q, k_pool, v_pool, block_table, seq_lens, page_size: int, o, lse, scale: float,
+                      workspace: torch.Tensor, stream=None) -> None:
+    """One decode step over a paged KV cache (shapes as in include/attn_b200.h)."""
+    lib = load_library()
+    S, Hq, d = q.shape
+    num_pages, Hkv, ps, d2 = k_pool.shape
+    if ps != page_size or d2 != d or tuple(v_pool.shape) != tuple(k_pool.shape):
+        raise ValueError("pools must be [num_pages, Hkv, page_size, d]")
+    if block_table.dim() != 2 or block_table.shape[0] != S:
+        raise ValueError("block_table must be [num_seqs, max_pages_per_seq]")
+    max_pages = block_table.shape[1]
+    st = lib.attn_decode_paged(
+        _dev(q, "q", torch.bfloat16, 3), _dev(k_pool, "k_pool", torch.bfloat16, 4),
+        _dev(v_pool, "v_pool", torch.bfloat16, 4), _dev(block_table, "block_table", torch.int32, 2),
+        _dev(seq_lens, "seq_lens", torch.int32, 1), page_size, _dev(o, "o", torch.bfloat16, 3),
+        None if lse is None else _dev(lse, "lse", torch.float32, 2), S, Hq, Hkv, d, num_pages, max_pages,
+        float(scale), _dev(workspace, "workspace", workspace.dtype), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check(st, "attn_decode_paged")
+
+
+def attn_get_device_status(stream=None) -> int:
+    """Synchronises the stream; returns and clears the first fault a kernel latched."""
+    return int(load_library().attn_get_device_status(_stream(stream)))
+
+
+def attn_debug_watchdog(timeout_ns: int, stream=None) -> None:
+    _check(load_library().attn_debug_watchdog(int(timeout_ns), _stream(stream)), "attn_debug_watchdog")
+
+
+def attn_status_string(status: int) -> str:
+    return load_library().attn_status_string(int(status)).decode()

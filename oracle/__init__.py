@@ -1,0 +1,16 @@
+"""fp64 CPU oracle for exact attention and paged-KV decode.
+
+Test infrastructure: used only by the tests, the smoke check and the
+benchmark's CPU-baseline leg.  It shares no code with the CUDA library.
+"""
+
+from .attention import (  # noqa: F401
+    as_f64,
+    attention,
+    attention_head,
+    attention_rows,
+    causal_visible,
+    decode_paged,
+    gather_pages,
+    kv_head_of,
+)
