@@ -1,0 +1,324 @@
+// attn_api.cu — the C ABI declared in include/attn_b200.h.
+//
+// Host side only: argument checks, TMA tensor-map encoding, launch configuration.
+// Every step of the computation runs in the kernels of prefill_sm100.cuh and
+// decode_sm100.cuh.  The whole library is this one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn_b200.h"
+#include "decode_sm100.cuh"
+#include "prefill_sm100.cuh"
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;  // 1 s per pipeline wait
+constexpr int kMaxDevices = 64;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor map over [outer, rows, inner] with a {64, box_rows, 1} box, 128-byte
+// swizzle and zero fill outside the tensor (rows past `rows` read as zero).
+bool encode_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
+               uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {inner, rows, outer};
+  cuuint64_t strides[2] = {inner * 2, rows * inner * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+// Raises the dynamic shared-memory limit of each kernel once per device.
+template <typename K>
+bool ensure_smem(K kernel, int bytes, int slot) {
+  static std::mutex mu;
+  static std::atomic<uint64_t> done[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return false;
+  const uint64_t bit = 1ull << slot;
+  if (done[dev].load(std::memory_order_acquire) & bit) return true;
+  std::lock_guard<std::mutex> g(mu);
+  if (done[dev].load() & bit) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  done[dev].fetch_or(bit, std::memory_order_release);
+  return true;
+}
+
+int sm_count() {
+  static std::atomic<int> cache[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  int v = cache[dev].load();
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cache[dev].store(v);
+  }
+  return v;
+}
+
+attn_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D>
+attn_status launch_prefill(attn::FwdArgs& a, cudaStream_t st) {
+  if constexpr (D <= 128) {
+    using C = attn::PingPongCfg<D>;
+    auto k = attn::attn_fwd_pingpong_kernel<D>;
+    if (!ensure_smem(k, C::SMEM, D == 64 ? 0 : 1)) return ATTN_ERR_CUDA;
+    const long long qp = (a.n_qtiles + 1) / 2;
+    const long long units = a.pair_heads ? (long long)a.B * (a.Hq / 2) * a.n_qtiles : (long long)a.B * a.Hq * qp;
+    if (units <= 0 || units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    a.n_units = (int)units;
+    k<<<(unsigned)units, C::THREADS, C::SMEM, st>>>(a);
+  } else {
+    using C = attn::SingleCfg<D>;
+    auto k = attn::attn_fwd_single_kernel<D>;
+    if (!ensure_smem(k, C::SMEM, 2)) return ATTN_ERR_CUDA;
+    const long long units = (long long)a.B * a.Hq * a.n_qtiles;
+    if (units <= 0 || units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    a.n_units = (int)units;
+    k<<<(unsigned)units, C::THREADS, C::SMEM, st>>>(a);
+  }
+  return launch_status();
+}
+
+template <int D>
+attn_status launch_decode(attn::DecArgs& a, cudaStream_t st, long long max_items) {
+  using C = attn::DecCfg<D>;
+  auto ks = attn::attn_decode_split_kernel<D>;
+  const int slot = D == 64 ? 3 : (D == 128 ? 4 : 5);
+  if (!ensure_smem(ks, C::SMEM, slot)) return ATTN_ERR_CUDA;
+  attn::attn_decode_plan_kernel<<<1, 1024, 0, st>>>(a.seq_lens, a.S, a.max_pages * a.page_size, a.chunk_prefix);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  long long grid = (long long)sm_count() * C::CTAS_PER_SM;
+  if (grid > max_items) grid = max_items;
+  if (grid < 1) grid = 1;
+  ks<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  const long long warps = (long long)a.S * a.Hq;
+  const long long blocks = (warps * 32 + 255) / 256;
+  attn::attn_decode_merge_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(a);
+  return launch_status();
+}
+
+struct DecodeLayout {
+  size_t off_prefix, off_part_o, off_part_lse, total;
+  int max_chunks;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool decode_layout(int S, int Hq, int d, int max_pages, int page_size, DecodeLayout* L) {
+  if (S < 0 || Hq <= 0 || d <= 0 || max_pages <= 0 || page_size <= 0) return false;
+  const long long max_tokens = (long long)max_pages * page_size;
+  if (max_tokens > 0x7fffffffLL) return false;
+  L->max_chunks = (int)((max_tokens + attn::kDecChunkTok - 1) / attn::kDecChunkTok);
+  const size_t parts = (size_t)S * L->max_chunks * Hq;
+  L->off_prefix = 0;
+  L->off_part_o = align256((size_t)(S + 1) * 4);
+  L->off_part_lse = L->off_part_o + align256(parts * d * 4);
+  L->total = L->off_part_lse + align256(parts * 4);
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_abi_version(void) { return 1; }
+
+const char* attn_status_string(int s) {
+  switch (s) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_ALIGNMENT: return "ATTN_ERR_ALIGNMENT";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "ATTN_ERR_DEVICE_TIMEOUT";
+    case ATTN_ERR_BAD_PAGE: return "ATTN_ERR_BAD_PAGE";
+    case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE";
+    default: return "ATTN_STATUS_UNKNOWN";
+  }
+}
+
+attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, int o_dtype, float* lse, int B,
+                        int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, void* stream) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (o_dtype != ATTN_DTYPE_BF16 && o_dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || Nq == 0) return ATTN_OK;
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (q == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (Nk > 0 && (k == nullptr || v == nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(o, 16) || (Nk > 0 && (!aligned(k, 16) || !aligned(v, 16))) ||
+      (lse != nullptr && !aligned(lse, 4)))
+    return ATTN_ERR_ALIGNMENT;
+  if ((long long)B * Hq > 0x7fffffffLL || (long long)B * Hkv > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int o_f32 = o_dtype == ATTN_DTYPE_F32;
+
+  if (Nk == 0) {  // no key is visible to any row
+    const size_t rows = (size_t)B * Hq * Nq;
+    attn::attn_fwd_empty_kernel<<<592, 256, 0, st>>>(o, lse, rows, d, o_f32);
+    return launch_status();
+  }
+
+  attn::FwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  const uint32_t bn = d <= 128 ? 128 : 64;
+  if (!encode_3d(&a.tm_q, q, d, Nq, (uint64_t)B * Hq, 128) || !encode_3d(&a.tm_k, k, d, Nk, (uint64_t)B * Hkv, bn) ||
+      !encode_3d(&a.tm_v, v, d, Nk, (uint64_t)B * Hkv, bn))
+    return ATTN_ERR_CUDA;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Nq = Nq;
+  a.Nk = Nk;
+  a.group = Hq / Hkv;
+  a.causal = causal;
+  a.o_f32 = o_f32;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.pair_heads = (a.group % 2 == 0) ? 1 : 0;
+  a.n_qtiles = (Nq + 127) / 128;
+  a.timeout_ns = kDefaultTimeoutNs;
+  switch (d) {
+    case 64: return launch_prefill<64>(a, st);
+    case 128: return launch_prefill<128>(a, st);
+    default: return launch_prefill<256>(a, st);
+  }
+}
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                     int Nq, int Nk, int d, float scale, int causal, void* stream) {
+  return attn_fwd_ex(q, k, v, o, ATTN_DTYPE_BF16, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream);
+}
+
+size_t attn_decode_paged_workspace_size(int num_seqs, int Hq, int Hkv, int d, int max_pages_per_seq,
+                                        int page_size) {
+  if (Hkv <= 0 || Hq <= 0 || Hq % Hkv != 0) return 0;
+  if (d != 64 && d != 128 && d != 256) return 0;
+  if (page_size != 16 && page_size != 32 && page_size != 64) return 0;
+  DecodeLayout L;
+  if (!decode_layout(num_seqs, Hq, d, max_pages_per_seq, page_size, &L)) return 0;
+  return L.total;
+}
+
+attn_status attn_decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_table,
+                              const int32_t* seq_lens, int page_size, void* o, float* lse, int num_seqs, int Hq,
+                              int Hkv, int d, int num_pages, int max_pages_per_seq, float scale, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (num_seqs < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || num_pages < 0 || max_pages_per_seq <= 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  if (page_size != 16 && page_size != 32 && page_size != 64) return ATTN_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return ATTN_OK;
+  if (q == nullptr || o == nullptr || block_table == nullptr || seq_lens == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (num_pages > 0 && (k_pool == nullptr || v_pool == nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 4) || !aligned(o, 4) || !aligned(block_table, 4) || !aligned(seq_lens, 4) ||
+      (lse != nullptr && !aligned(lse, 4)) || (num_pages > 0 && (!aligned(k_pool, 16) || !aligned(v_pool, 16))))
+    return ATTN_ERR_ALIGNMENT;
+  if ((long long)num_pages * Hkv > 0x7fffffffLL || (long long)num_seqs * Hq > 0x7fffffffLL)
+    return ATTN_ERR_INVALID_ARG;
+  DecodeLayout L;
+  if (!decode_layout(num_seqs, Hq, d, max_pages_per_seq, page_size, &L)) return ATTN_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < L.total) return ATTN_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return ATTN_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  attn::DecArgs a;
+  std::memset(&a, 0, sizeof(a));
+  // an empty pool still needs a valid descriptor; no page id can then be in range
+  const void* kp = num_pages > 0 ? k_pool : q;
+  const void* vp = num_pages > 0 ? v_pool : q;
+  const uint64_t outer = num_pages > 0 ? (uint64_t)num_pages * Hkv : 1;
+  const uint64_t rows = num_pages > 0 ? (uint64_t)page_size : 1;
+  if (num_pages > 0) {
+    if (!encode_3d(&a.tm_k, kp, d, rows, outer, attn::kDecTok) || !encode_3d(&a.tm_v, vp, d, rows, outer, attn::kDecTok))
+      return ATTN_ERR_CUDA;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.block_table = block_table;
+  a.seq_lens = seq_lens;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.chunk_prefix = reinterpret_cast<int*>(ws + L.off_prefix);
+  a.part_o = reinterpret_cast<float*>(ws + L.off_part_o);
+  a.part_lse = reinterpret_cast<float*>(ws + L.off_part_lse);
+  a.S = num_seqs;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.group = Hq / Hkv;
+  a.n_hgroups = (a.group + 15) / 16;
+  a.page_size = page_size;
+  a.num_pages = num_pages;
+  a.max_pages = max_pages_per_seq;
+  a.max_chunks = L.max_chunks;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.timeout_ns = kDefaultTimeoutNs;
+  const long long max_items = (long long)num_seqs * L.max_chunks * Hkv * a.n_hgroups;
+  if (max_items > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  switch (d) {
+    case 64: return launch_decode<64>(a, st, max_items);
+    case 128: return launch_decode<128>(a, st, max_items);
+    default: return launch_decode<256>(a, st, max_items);
+  }
+}
+
+attn_status attn_debug_watchdog(uint64_t timeout_ns, void* stream) {
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;
+  attn::attn_watchdog_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+  return launch_status();
+}
+
+attn_status attn_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, attn::g_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(attn::g_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  return static_cast<attn_status>(v);
+}
+
+}  // extern "C"

@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Benchmark of the attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  1. prefill attention forward on the GQA causal 2K workload
+     (B=4, Hq=32, Hkv=8, Nq=Nk=2048, d=128, bf16, causal), then
+  2. one paged-KV decode step on the 64-sequence workload
+     (Hq=64, Hkv=8, d=128, 16-token pages, lengths uniform in [512, 32768]).
+The decode streams about 4.6 GB of cached K/V, far more than the 126 MB L2, so every
+prefill launch starts with a cold L2 for its own inputs.
+
+Printed (rank 0, one JSON line): prefill TFLOP/s as `value` (causal FLOPs counted as
+half of 4*B*Hq*Nq*Nk*d), the decode KV-read GB/s in `decode`, roofline fractions
+against MEASURED_PEAKS.json, the end-to-end figure through the public API with host
+buffers (`e2e`), the fp64 CPU oracle timed on a bounded sample (`cpu_baseline`), and
+the SM clocks sampled during the run.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload serving_step|gqa_causal_16k|peaked_mha_d256|tiny_mha_d64]
+
+With N > 1 (launched by torchrun, one process per GPU) every rank runs its own
+independent copy of the workload (weak scaling: the path shards into independent
+problems and has no exchange step); times are the maximum over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from attn_fwd_05_b200 import counts, synth  # noqa: E402
+
+METRIC = "attn fwd TFLOPS & % of BF16 tensor peak; paged decode KV-read GB/s & % HBM"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="serving_step",
+                   choices=["serving_step", "gqa_causal_16k", "peaked_mha_d256", "tiny_mha_d64", "gqa_causal_2k"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="bounded CPU-baseline sample length")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- distributed
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.on = self.world > 1
+
+    def init(self, backend="nccl"):
+        if self.on:
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", self.local) if backend == "nccl" else None)
+
+    def barrier(self):
+        if self.on:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.on:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=torch.device("cuda", self.local))
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.on:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling in the background while the GPU works."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            uuid = str(device_index)
+        self.uuid = uuid
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 10:
+                    rows.append(parts)
+        os.unlink(self.path)
+        busy = [r for r in rows if _num(r[4]) and _num(r[4]) > 0] or rows
+        sm = [_num(r[1]) for r in busy if _num(r[1])]
+        mx = [_num(r[2]) for r in busy if _num(r[2])]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in busy for i in range(4) if r[6 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(busy),
+                "power_w_max": max((_num(r[3]) or 0.0) for r in busy) if busy else None}
+
+
+def _num(s):
+    try:
+        return float(s)
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def prefill_shape(name: str):
+    return synth.WORKLOADS["gqa_causal_2k" if name == "serving_step" else name]
+
+
+def make_prefill(shape, seed, dev):
+    q, k, v = synth.prefill_inputs(shape, seed)
+    o = torch.empty((shape.B, shape.Hq, shape.Nq, shape.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((shape.B, shape.Hq, shape.Nq), dtype=torch.float32, device=dev)
+    return {"host": (q, k, v), "dev": (q.to(dev), k.to(dev), v.to(dev)), "o": o, "lse": lse}
+
+
+def make_decode(seed, dev):
+    import attn_fwd_05_b200 as ab
+    s = synth.WORKLOADS["paged_decode_gqa"]
+    kv = synth.decode_inputs(s, seed)
+    S = s.S
+    ws_bytes = ab.attn_decode_paged_workspace_size(S, s.Hq, s.Hkv, s.d, kv.max_pages_per_seq, s.page_size)
+    return {
+        "kv": kv, "shape": s,
+        "q": kv.q.to(dev), "k_pool": kv.k_pool.to(dev), "v_pool": kv.v_pool.to(dev),
+        "table": kv.block_table.to(dev), "lens": kv.seq_lens.to(dev),
+        "o": torch.empty((S, s.Hq, s.d), dtype=torch.bfloat16, device=dev),
+        "lse": torch.empty((S, s.Hq), dtype=torch.float32, device=dev),
+        "ws": torch.empty(ws_bytes, dtype=torch.uint8, device=dev),
+        "kv_bytes": counts.decode_kv_bytes(kv.seq_lens.tolist(), s.Hkv, s.d),
+    }
+
+
+# ----------------------------------------------------------------------------- CPU oracle (baseline / reference arm)
+
+def oracle_prefill_sample(shape, q, k, v, seconds: float, max_heads=None):
+    """Time the fp64 oracle on whole heads of the workload until `seconds` have passed."""
+    from oracle import attention
+    threads = os.cpu_count() or 1
+    scale = synth.default_scale(shape.d)
+    G = shape.Hq // shape.Hkv
+    heads = [(b, h) for b in range(shape.B) for h in range(shape.Hq)]
+    if max_heads:
+        heads = heads[:max_heads]
+    done = 0
+    t0 = time.perf_counter()
+    i = 0
+    while i < len(heads):
+        batch = heads[i:i + threads]
+        for b, h in batch:
+            pass
+        qs = torch.stack([q[b, h] for b, h in batch])[None]
+        ks = torch.stack([k[b, h // G] for b, h in batch])[None]
+        vs = torch.stack([v[b, h // G] for b, h in batch])[None]
+        attention(qs, ks, vs, scale, shape.causal, threads=threads)
+        done += len(batch)
+        i += len(batch)
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    flops = counts.prefill_flops(1, done, shape.Nq, shape.Nk, shape.d, shape.causal)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} of {len(heads)} (batch, head) pairs of the workload, {dt:.1f} s, fp64 numpy"}
+
+
+def oracle_decode_sample(dec, seconds: float):
+    from oracle import decode_paged
+    kv = dec["kv"]
+    s = dec["shape"]
+    scale = synth.default_scale(s.d)
+    t0 = time.perf_counter()
+    seqs = []
+    for n in range(s.S):
+        decode_paged(kv.q, kv.k_pool, kv.v_pool, kv.block_table, kv.seq_lens, s.page_size, scale, seqs=[n])
+        seqs.append(n)
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    nbytes = counts.decode_kv_bytes([int(kv.seq_lens[i]) for i in seqs], s.Hkv, s.d)
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{len(seqs)} of {s.S} sequences, {dt:.1f} s, fp64 numpy"}
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_reference(args, dist):
+    """The oracle, as it stands, on the host cores, on the same config and metric."""
+    if dist.rank != 0:
+        return 0
+    shape = prefill_shape(args.workload)
+    q, k, v = synth.prefill_inputs(shape, synth.workload_seed(
+        "gqa_causal_2k" if args.workload == "serving_step" else args.workload))
+    per_step = max(0.5, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_prefill_sample(shape, q, k, v, per_step, max_heads=os.cpu_count())
+    vals, secs = [], []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r = oracle_prefill_sample(shape, q, k, v, per_step, max_heads=os.cpu_count())
+        vals.append(r["value"])
+    total = time.perf_counter() - t0
+    value = statistics.mean(vals) if vals else 0.0
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(args, shape),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"per step: {os.cpu_count()} (batch, head) pairs of the prefill workload"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(args, shape):
+    cfg = {"workload": "gqa_causal_2k prefill + paged_decode_gqa decode" if args.workload == "serving_step"
+           else args.workload,
+           "prefill": {"B": shape.B, "Hq": shape.Hq, "Hkv": shape.Hkv, "Nq": shape.Nq, "Nk": shape.Nk, "d": shape.d,
+                       "causal": shape.causal, "qk_std": shape.qk_std}}
+    if args.workload == "serving_step":
+        s = synth.WORKLOADS["paged_decode_gqa"]
+        cfg["decode"] = {"seqs": s.S, "Hq": s.Hq, "Hkv": s.Hkv, "d": s.d, "page_size": s.page_size,
+                         "len_range": [s.len_lo, s.len_hi]}
+        cfg["l2"] = "inputs larger than L2: each step's 4.6 GB decode KV stream evicts the prefill inputs"
+    else:
+        cfg["l2"] = "L2 flushed between steps by writing a 256 MB buffer"
+    cfg["parallelism"] = f"independent replicas x{args.gpus} (no data-path collective)"
+    return cfg
+
+
+def run_ours(args, dist):
+    import attn_fwd_05_b200 as ab
+    ab.load_library()
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    shape = prefill_shape(args.workload)
+    seed = synth.workload_seed("gqa_causal_2k" if args.workload == "serving_step" else args.workload)
+    pre = make_prefill(shape, seed + 7919 * dist.rank, dev)
+    dec = make_decode(synth.workload_seed("paged_decode_gqa") + 7919 * dist.rank, dev) \
+        if args.workload == "serving_step" else None
+    flush = None if dec is not None else torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    scale = synth.default_scale(shape.d)
+    flops = counts.prefill_flops(shape.B, shape.Hq, shape.Nq, shape.Nk, shape.d, shape.causal)
+    stream = torch.cuda.current_stream(dev)
+
+    qd, kd, vd = pre["dev"]
+
+    def prefill():
+        ab.attn_fwd(qd, kd, vd, pre["o"], pre["lse"], shape.causal, scale, stream)
+
+    def decode():
+        ab.attn_decode_paged(dec["q"], dec["k_pool"], dec["v_pool"], dec["table"], dec["lens"],
+                             dec["shape"].page_size, dec["o"], dec["lse"], scale, dec["ws"], stream)
+
+    clocks = ClockSampler(dist.local)
+    clocks.start()
+    for _ in range(args.warmup):
+        prefill()
+        if dec is not None:
+            decode()
+        else:
+            flush.zero_()
+    torch.cuda.synchronize(dev)
+    st = ab.attn_get_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"kernel fault during warm-up: {ab.attn_status_string(st)}")
+
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3 * K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_start.record(stream)
+    for i in range(K):
+        if dec is None:
+            flush.zero_()
+        ev[3 * i].record(stream)
+        prefill()
+        ev[3 * i + 1].record(stream)
+        if dec is not None:
+            decode()
+        ev[3 * i + 2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clk = clocks.stop()
+    st = ab.attn_get_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"kernel fault in the timed region: {ab.attn_status_string(st)}")
+
+    pre_ms = [ev[3 * i].elapsed_time(ev[3 * i + 1]) for i in range(K)]
+    dec_ms = [ev[3 * i + 1].elapsed_time(ev[3 * i + 2]) for i in range(K)] if dec is not None else []
+    total_ms = t_start.elapsed_time(t_end)
+    pre_sum = dist.max(sum(pre_ms))
+    dec_sum = dist.max(sum(dec_ms)) if dec is not None else 0.0
+    total_ms = dist.max(total_ms)
+    N = dist.world
+
+    prefill_tflops = N * flops * K / (pre_sum * 1e-3) / 1e12
+    avg_pre_ms = sum(pre_ms) / K
+    achieved = flops / (avg_pre_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": prefill_tflops,
+        "unit": "TFLOP/s",
+        "n_gpus": N,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": config_block(args, shape),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops (burst cuBLAS); "
+                                    f"frac of sustained {achieved / peaks['bf16_tflops_sustained']:.3f}",
+                     "kernel": "attn_fwd_pingpong_kernel<128>" if shape.d <= 128 else "attn_fwd_single_kernel<256>",
+                     "median_ms": statistics.median(pre_ms)},
+        "gpu_launches": K * (1 + (3 if dec is not None else 0)),
+        "clocks": clk,
+    }
+    if dec is not None:
+        kvb = dec["kv_bytes"]
+        avg_dec_ms = sum(dec_ms) / K
+        gbs = kvb / (avg_dec_ms * 1e-3) / 1e9
+        line["decode"] = {
+            "metric": "paged decode KV-read GB/s", "value": N * kvb * K / (dec_sum * 1e-3) / 1e9, "unit": "GB/s",
+            "kv_bytes_per_step": kvb, "median_ms": statistics.median(dec_ms),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                         "peak_source": f"{peak_src} hbm_gbs (copy)",
+                         "kernels": "attn_decode_plan + attn_decode_split_kernel<128> + attn_decode_merge_kernel<128>"},
+        }
+
+    if not args.no_e2e:
+        line["e2e"] = e2e_prefill(args, ab, pre, shape, scale, flops, dev, stream, dist)
+    if dist.rank == 0 and N == 1 and not args.no_cpu_baseline:
+        q, k, v = pre["host"]
+        line["cpu_baseline"] = oracle_prefill_sample(shape, q, k, v, args.cpu_seconds)
+        if dec is not None:
+            line["decode"]["cpu_baseline"] = oracle_decode_sample(dec, max(2.0, args.cpu_seconds / 3))
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def e2e_prefill(args, ab, pre, shape, scale, flops, dev, stream, dist):
+    """Same metric through the public API with host buffers: H2D of q, k, v from pinned
+    memory, attn_fwd, D2H of o and lse, all inside the timed region."""
+    qh, kh, vh = (t.pin_memory() for t in pre["host"])
+    oh = torch.empty(pre["o"].shape, dtype=torch.bfloat16).pin_memory()
+    lh = torch.empty(pre["lse"].shape, dtype=torch.float32).pin_memory()
+    qd = torch.empty_like(qh, device=dev)
+    kd = torch.empty_like(kh, device=dev)
+    vd = torch.empty_like(vh, device=dev)
+
+    def step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        ab.attn_fwd(qd, kd, vd, pre["o"], pre["lse"], shape.causal, scale, stream)
+        oh.copy_(pre["o"], non_blocking=True)
+        lh.copy_(pre["lse"], non_blocking=True)
+
+    K = max(3, min(args.steps, 20))
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    a.record(stream)
+    for _ in range(K):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = dist.max(a.elapsed_time(b))
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * 2 + lh.numel() * 4
+    return {"value": dist.world * flops * K / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K}
+
+
+def main():
+    args = parse()
+    dist = Dist()
+    if args.impl == "reference":
+        return run_reference(args, dist)
+    dist.init("nccl")
+    try:
+        return run_ours(args, dist)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

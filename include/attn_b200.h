@@ -1,0 +1,167 @@
+/*
+ * attn_b200.h — exact scaled-dot-product attention on one NVIDIA B200 (sm_100a).
+ *
+ * What is computed
+ *   O = softmax(scale * Q K^T + mask) V, row by row, exactly up to floating-point
+ *   rounding.  The formula is the one of the polydesk.ai glossary page
+ *   "FlashAttention" (section "Le goulot d'étranglement de l'attention standard")
+ *   and of ranksignal.fr, "FlashAttention et PagedAttention : à quoi servent-elles ?"
+ *   (section "FlashAttention : calculer sur le plan de travail").  The computation is
+ *   tiled with an online softmax (running row maximum and sum of exponentials,
+ *   rescaled per tile; same glossary page, section "L'idée clé : IO-awareness"), so the
+ *   N x N score matrix never reaches device memory.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers marked "device" must point to device memory of the current CUDA device;
+ *     the library reads and writes them only from kernels on `stream`.
+ *   - Every tensor is dense and row-major (the last dimension is contiguous).
+ *   - bf16 tensors are IEEE bfloat16 stored as 16-bit words.
+ *   - Device pointers passed to the tensor-memory-accelerator (TMA) loads (q, k, v,
+ *     k_pool, v_pool) must be 16-byte aligned; every other device pointer must be
+ *     aligned to its element size, and o to 16 bytes.
+ *   - The caller owns every buffer.  attn_fwd and attn_fwd_ex allocate nothing;
+ *     attn_decode_paged takes all its scratch from the caller's `workspace`.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
+ *     stream) and never synchronise.  Entry points are thread-safe.
+ *   - Errors are returned as attn_status codes; no exception crosses this interface.
+ *     Argument checks run on the host before any launch; a call that fails them has
+ *     launched nothing and touched no buffer.  Faults found by a kernel (a page id
+ *     outside the pool, a pipeline wait that ran past its time limit) are latched in
+ *     a per-device status word and reported by attn_get_device_status.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum attn_status {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,     /* null pointer, negative size, Hq % Hkv != 0, bad scale ... */
+  ATTN_ERR_UNSUPPORTED = 2,     /* a head dimension or page size this build has no kernel for */
+  ATTN_ERR_ALIGNMENT = 3,       /* a device pointer breaks the alignment rule above */
+  ATTN_ERR_CUDA = 4,            /* a CUDA runtime or driver call failed */
+  ATTN_ERR_DEVICE_TIMEOUT = 5,  /* a kernel's bounded pipeline wait gave up */
+  ATTN_ERR_BAD_PAGE = 6,        /* a block-table entry in use lies outside [0, num_pages) */
+  ATTN_ERR_WORKSPACE = 7        /* workspace null or smaller than attn_decode_paged_workspace_size */
+} attn_status;
+
+typedef enum attn_dtype {
+  ATTN_DTYPE_BF16 = 0,
+  ATTN_DTYPE_F32 = 1
+} attn_dtype;
+
+/* Version of this interface; bumped whenever a signature changes. */
+int attn_abi_version(void);
+
+/*
+ * attn_fwd — prefill attention forward.
+ *
+ * Source: the formula above; causal masking is the triangular mask the
+ * patricehuetz.fr page "Flash Attention : pourquoi ton GPU utilise 85% de VRAM"
+ * (section "Cas 2 : masques d'attention custom") names as the supported case, and
+ * grouped-query heads are those of analyticslegends.ai, "Variantes d'attention"
+ * (glossary entry GQA: H_q query heads share H_kv < H_q K/V groups).
+ *
+ *   q    device, bf16 [B, Hq,  Nq, d]
+ *   k    device, bf16 [B, Hkv, Nk, d]
+ *   v    device, bf16 [B, Hkv, Nk, d]
+ *   o    device, bf16 [B, Hq,  Nq, d]            (written)
+ *   lse  device, fp32 [B, Hq,  Nq] or NULL       (written when not NULL)
+ *        lse = ln sum_j exp(scale * q.k_j) over the visible keys j.
+ *   B, Hq, Hkv, Nq, Nk >= 0 (B, Hq, Hkv >= 1 when Nq > 0);  Hq % Hkv == 0;
+ *   query head h reads K/V head h / (Hq / Hkv).
+ *   d    head dimension: 64, 128 or 256.
+ *   scale > 0 and finite (1/sqrt(d) for the usual softmax temperature).
+ *   causal  0: every key visible.  1: key j visible to query i iff
+ *           j <= i + (Nk - Nq) (mask aligned to the bottom-right corner).
+ *   A query row with no visible key gets O = 0 and lse = -inf.
+ *   Nq == 0 is a no-op.  Limits: B*Hq and B*Hkv < 2^31, Nq and Nk < 2^31.
+ * Returns ATTN_OK once the kernel is enqueued.
+ */
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                     int causal, void* stream);
+
+/*
+ * attn_fwd_ex — attn_fwd with a choice of output type: the same kernel, whose
+ * epilogue writes O as bf16 (o_dtype = ATTN_DTYPE_BF16) or as fp32
+ * (ATTN_DTYPE_F32, o is then fp32 [B, Hq, Nq, d]).  The fp32 form exposes the
+ * kernel's accumulator before the final bf16 rounding.
+ */
+attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, int o_dtype,
+                        float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                        int causal, void* stream);
+
+/*
+ * attn_decode_paged_workspace_size — bytes of scratch attn_decode_paged needs for
+ * these sizes (fp32 partial outputs and partial log-sum-exps of the split-K pass).
+ * Returns 0 for sizes attn_decode_paged would reject.
+ */
+size_t attn_decode_paged_workspace_size(int num_seqs, int Hq, int Hkv, int d,
+                                        int max_pages_per_seq, int page_size);
+
+/*
+ * attn_decode_paged — one decode step over a paged KV cache.
+ *
+ * Source: ranksignal.fr, "FlashAttention et PagedAttention : à quoi servent-elles ?",
+ * sections "Le cache KV, ce locataire qui grossit" (the new token attends to the kept
+ * keys and values of all earlier tokens) and "PagedAttention : ranger par pages plutôt
+ * que d'un seul tenant" (the cache lives in fixed-size pages reached through a table;
+ * paging changes where data lives, not what is computed).
+ *
+ *   q            device, bf16 [num_seqs, Hq, d]: one query token per sequence
+ *   k_pool       device, bf16 [num_pages, Hkv, page_size, d]
+ *   v_pool       device, bf16 [num_pages, Hkv, page_size, d]
+ *   block_table  device, int32 [num_seqs, max_pages_per_seq]: entry i of row s is the
+ *                pool page holding tokens [i*page_size, (i+1)*page_size) of sequence s;
+ *                entries past ceil(seq_lens[s]/page_size) are never read.
+ *   seq_lens     device, int32 [num_seqs]: cached tokens per sequence, each in
+ *                [0, max_pages_per_seq*page_size]; the query attends to all of them.
+ *   o            device, bf16 [num_seqs, Hq, d]   (written)
+ *   lse          device, fp32 [num_seqs, Hq] or NULL (written when not NULL)
+ *   page_size    16, 32 or 64;  d: 64, 128 or 256;  Hq % Hkv == 0 and Hq/Hkv <= 16.
+ *   workspace    device scratch of at least attn_decode_paged_workspace_size(...) bytes,
+ *                owned by the caller; its contents need no initialisation and are
+ *                overwritten.  Two calls in flight at once need two workspaces.
+ *   A sequence of length 0 gets O = 0 and lse = -inf.  A block-table entry in use that
+ *   lies outside [0, num_pages) is not read: the kernel skips that page and latches
+ *   ATTN_ERR_BAD_PAGE (see attn_get_device_status).
+ * Launches two kernels on `stream`: the split-K pass over pages, then the merge of the
+ * partial results by their log-sum-exp.
+ */
+attn_status attn_decode_paged(const void* q, const void* k_pool, const void* v_pool,
+                              const int32_t* block_table, const int32_t* seq_lens,
+                              int page_size, void* o, float* lse, int num_seqs, int Hq,
+                              int Hkv, int d, int num_pages, int max_pages_per_seq,
+                              float scale, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
+ * attn_get_device_status — synchronises `stream`, then returns and clears the first
+ * fault a kernel of this library latched on the current device since the last call
+ * (ATTN_OK if none).  ATTN_ERR_CUDA if the synchronisation itself fails.
+ */
+attn_status attn_get_device_status(void* stream);
+
+/*
+ * attn_debug_watchdog — failure-path check, computes nothing.  Launches one CTA on
+ * `stream` whose single thread waits on a pipeline barrier that nothing completes;
+ * the bounded wait every kernel of this library uses gives up after timeout_ns
+ * (1 ns .. 10 s) and latches ATTN_ERR_DEVICE_TIMEOUT, which attn_get_device_status
+ * then reports.  The kernel exits normally; the device stays usable.
+ */
+attn_status attn_debug_watchdog(uint64_t timeout_ns, void* stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* attn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */
