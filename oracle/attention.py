@@ -187,8 +187,16 @@ class _nullctx:
 # "PagedAttention : ranger par pages plutôt que d'un seul tenant")
 # ----------------------------------------------------------------------------
 
-def gather_pages(pool: np.ndarray, table_row: np.ndarray, seq_len: int, page_size: int) -> np.ndarray:
-    """Rebuild one sequence's contiguous cache [Hkv, seq_len, d] from its pages.
+def _pages_f64(pool, ids: np.ndarray) -> np.ndarray:
+    """pool[ids] widened to float64; only the selected pages are converted."""
+    if hasattr(pool, "detach"):
+        import torch
+        return as_f64(pool[torch.as_tensor(ids, dtype=torch.long)])
+    return np.asarray(pool)[ids].astype(np.float64)
+
+
+def gather_pages(pool, table_row, seq_len: int, page_size: int) -> np.ndarray:
+    """Rebuild one sequence's contiguous cache [Hkv, seq_len, d] (float64) from its pages.
 
     pool: [num_pages, Hkv, page_size, d]; entry i of the table row holds tokens
     [i*page_size, (i+1)*page_size).  Raises on a page id outside the pool.
@@ -197,7 +205,7 @@ def gather_pages(pool: np.ndarray, table_row: np.ndarray, seq_len: int, page_siz
     ids = np.asarray(table_row[:npages], dtype=np.int64)
     if npages and (ids.min() < 0 or ids.max() >= pool.shape[0]):
         raise IndexError("block table entry outside the page pool")
-    pages = pool[ids]                                   # [npages, Hkv, page_size, d]
+    pages = _pages_f64(pool, ids)                       # [npages, Hkv, page_size, d]
     Hkv, d = pool.shape[1], pool.shape[3]
     seq = pages.transpose(1, 0, 2, 3).reshape(Hkv, npages * page_size, d)
     return seq[:, :seq_len]
@@ -212,12 +220,10 @@ def decode_paged(q, k_pool, v_pool, block_table, seq_lens, page_size: int, scale
     if given, in that order).
     """
     qf = as_f64(q)
-    kp = as_f64(k_pool)
-    vp = as_f64(v_pool)
     table = np.asarray(block_table.cpu() if hasattr(block_table, "cpu") else block_table)
     lens = np.asarray(seq_lens.cpu() if hasattr(seq_lens, "cpu") else seq_lens)
     S, Hq, d = qf.shape
-    Hkv = kp.shape[1]
+    Hkv = k_pool.shape[1]
     seqs = range(S) if seqs is None else list(seqs)
     O = np.zeros((len(seqs), Hq, d))
     L = np.full((len(seqs), Hq), -np.inf)
@@ -225,8 +231,8 @@ def decode_paged(q, k_pool, v_pool, block_table, seq_lens, page_size: int, scale
         ln = int(lens[s])
         if ln <= 0:
             continue
-        K = gather_pages(kp, table[s], ln, page_size)
-        V = gather_pages(vp, table[s], ln, page_size)
+        K = gather_pages(k_pool, table[s], ln, page_size)
+        V = gather_pages(v_pool, table[s], ln, page_size)
         for h in range(Hq):
             kv = kv_head_of(h, Hq, Hkv)
             o, l = attention_head(qf[s, h][None], K[kv], V[kv], scale, causal=False)
