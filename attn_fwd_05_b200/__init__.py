@@ -9,6 +9,7 @@ library is loaded on first use and a missing or unloadable library raises
 from .binding import (  # noqa: F401
     AttnError,
     attn_decode_paged,
+    attn_decode_paged_noalloc,
     attn_decode_paged_workspace_size,
     attn_fwd,
     attn_fwd_ex,

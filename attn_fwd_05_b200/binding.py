@@ -21,7 +21,7 @@ _LOCK = threading.Lock()
 ATTN_OK = 0
 STATUS_NAMES = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_ALIGNMENT",
                 4: "ATTN_ERR_CUDA", 5: "ATTN_ERR_DEVICE_TIMEOUT", 6: "ATTN_ERR_BAD_PAGE",
-                7: "ATTN_ERR_WORKSPACE"}
+                7: "ATTN_ERR_WORKSPACE", 8: "ATTN_ERR_TOO_LARGE"}
 DTYPE_BF16, DTYPE_F32 = 0, 1
 
 # exported symbol -> (restype, argtypes); mirrors include/attn_b200.h
@@ -34,6 +34,9 @@ SIGNATURES = {
     "attn_decode_paged_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
     "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P,
                                ctypes.c_size_t, _P]),
+    "attn_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float,
+                                       _P]),
+    "attn_decode_paged_noalloc_max_scratch": (ctypes.c_size_t, []),
     "attn_debug_watchdog": (_I, [ctypes.c_uint64, _P]),
     "attn_get_device_status": (_I, [_P]),
     "attn_status_string": (ctypes.c_char_p, [_I]),
@@ -151,6 +154,29 @@ def attn_decode_paged(q, k_pool, v_pool, block_table, seq_lens, page_size: int, 
         float(scale), _dev(workspace, "workspace", workspace.dtype), workspace.numel() * workspace.element_size(),
         _stream(stream))
     _check(st, "attn_decode_paged")
+
+
+def attn_decode_paged_noalloc(q, k_pool, v_pool, block_table, seq_lens, page_size: int, o, lse, scale: float,
+                              stream=None) -> None:
+    """attn_decode_paged without a workspace: the library's static scratch is used.
+
+    For callers that must not allocate device memory; raises AttnError with
+    ATTN_ERR_TOO_LARGE when the sizes need more scratch than the library holds.
+    """
+    lib = load_library()
+    S, Hq, d = q.shape
+    num_pages, Hkv, ps, d2 = k_pool.shape
+    if ps != page_size or d2 != d or tuple(v_pool.shape) != tuple(k_pool.shape):
+        raise ValueError("pools must be [num_pages, Hkv, page_size, d]")
+    if block_table.dim() != 2 or block_table.shape[0] != S:
+        raise ValueError("block_table must be [num_seqs, max_pages_per_seq]")
+    st = lib.attn_decode_paged_noalloc(
+        _dev(q, "q", torch.bfloat16, 3), _dev(k_pool, "k_pool", torch.bfloat16, 4),
+        _dev(v_pool, "v_pool", torch.bfloat16, 4), _dev(block_table, "block_table", torch.int32, 2),
+        _dev(seq_lens, "seq_lens", torch.int32, 1), page_size, _dev(o, "o", torch.bfloat16, 3),
+        None if lse is None else _dev(lse, "lse", torch.float32, 2), S, Hq, Hkv, d, num_pages,
+        block_table.shape[1], float(scale), _stream(stream))
+    _check(st, "attn_decode_paged_noalloc")
 
 
 def attn_get_device_status(stream=None) -> int:

@@ -157,6 +157,34 @@ bool decode_layout(int S, int Hq, int d, int max_pages, int page_size, DecodeLay
   return true;
 }
 
+// ---------------------------------------------------------------- static decode scratch
+//
+// Scratch of attn_decode_paged_noalloc: a fixed array in the library's device image,
+// so that the call needs no allocation.  Every device that loads the library holds it
+// until the process exits.  In host code `g_decode_scratch` is only a host-side stand-in
+// for the symbol; the device address comes from cudaGetSymbolAddress, once per device.
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) uint8_t g_decode_scratch[kStaticScratchBytes];
+
+// Device address of g_decode_scratch on the current device (looked up on the first
+// call for that device), or nullptr if the lookup failed.
+void* static_scratch_address() {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> g(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess) {
+      cudaGetLastError();  // reset the runtime error state so later calls are unaffected
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -173,6 +201,7 @@ const char* attn_status_string(int s) {
     case ATTN_ERR_DEVICE_TIMEOUT: return "ATTN_ERR_DEVICE_TIMEOUT";
     case ATTN_ERR_BAD_PAGE: return "ATTN_ERR_BAD_PAGE";
     case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE";
+    case ATTN_ERR_TOO_LARGE: return "ATTN_ERR_TOO_LARGE";
     default: return "ATTN_STATUS_UNKNOWN";
   }
 }
@@ -305,6 +334,27 @@ attn_status attn_decode_paged(const void* q, const void* k_pool, const void* v_p
     default: return launch_decode<256>(a, st, max_items);
   }
 }
+
+attn_status attn_decode_paged_noalloc(const void* q, const void* k_pool, const void* v_pool,
+                                      const int32_t* block_table, const int32_t* seq_lens, int page_size, void* o,
+                                      float* lse, int num_seqs, int Hq, int Hkv, int d, int num_pages,
+                                      int max_pages_per_seq, float scale, void* stream) {
+  // Same checks as attn_decode_paged, so that a rejected call never touches the device.
+  if (num_seqs < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || num_pages < 0 || max_pages_per_seq <= 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  if (page_size != 16 && page_size != 32 && page_size != 64) return ATTN_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return ATTN_OK;
+  const size_t need = attn_decode_paged_workspace_size(num_seqs, Hq, Hkv, d, max_pages_per_seq, page_size);
+  if (need == 0) return ATTN_ERR_INVALID_ARG;
+  if (need > kStaticScratchBytes) return ATTN_ERR_TOO_LARGE;
+  void* scratch = static_scratch_address();
+  if (scratch == nullptr) return ATTN_ERR_CUDA;
+  return attn_decode_paged(q, k_pool, v_pool, block_table, seq_lens, page_size, o, lse, num_seqs, Hq, Hkv, d,
+                           num_pages, max_pages_per_seq, scale, scratch, kStaticScratchBytes, stream);
+}
+
+size_t attn_decode_paged_noalloc_max_scratch(void) { return kStaticScratchBytes; }
 
 attn_status attn_debug_watchdog(uint64_t timeout_ns, void* stream) {
   if (timeout_ns == 0 || timeout_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;

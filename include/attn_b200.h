@@ -47,7 +47,9 @@ typedef enum attn_status {
   ATTN_ERR_CUDA = 4,            /* a CUDA runtime or driver call failed */
   ATTN_ERR_DEVICE_TIMEOUT = 5,  /* a kernel's bounded pipeline wait gave up */
   ATTN_ERR_BAD_PAGE = 6,        /* a block-table entry in use lies outside [0, num_pages) */
-  ATTN_ERR_WORKSPACE = 7        /* workspace null or smaller than attn_decode_paged_workspace_size */
+  ATTN_ERR_WORKSPACE = 7,       /* workspace null or smaller than attn_decode_paged_workspace_size */
+  ATTN_ERR_TOO_LARGE = 8        /* attn_decode_paged_noalloc: the call needs more scratch than the
+                                   library's static scratch holds */
 } attn_status;
 
 typedef enum attn_dtype {
@@ -140,6 +142,40 @@ attn_status attn_decode_paged(const void* q, const void* k_pool, const void* v_p
                               int Hkv, int d, int num_pages, int max_pages_per_seq,
                               float scale, void* workspace, size_t workspace_bytes,
                               void* stream);
+
+/*
+ * attn_decode_paged_noalloc — attn_decode_paged for callers that cannot allocate device
+ * memory.  (The pages have no counterpart of this entry point: it is a deployment aid.)
+ *
+ * Some callers may not call cudaMalloc at all: a plugin loaded into a host application
+ * that owns every byte of device memory through its own pool, or a serving loop that
+ * must never allocate on the request path (cudaMalloc can synchronise the device and
+ * its latency is unbounded).  This entry point takes no workspace and allocates
+ * nothing: its scratch is a static array of ATTN_DECODE_NOALLOC_MAX_SCRATCH bytes
+ * (32 MiB) inside the library, which every GPU that loads the library holds until the
+ * process exits.  The caller still passes all inputs and outputs, with the meaning,
+ * layout and alignment of attn_decode_paged, and gets the same results.
+ *
+ *   Returns ATTN_ERR_TOO_LARGE, having launched nothing, when
+ *   attn_decode_paged_workspace_size(num_seqs, Hq, Hkv, d, max_pages_per_seq,
+ *   page_size) exceeds that size; other argument errors are those of attn_decode_paged.
+ *   The first call on a device looks up the device address of the static array (a
+ *   cudaGetSymbolAddress on the current device); make that first call before any
+ *   stream capture.
+ *   Every call shares the one array and leaves its contents behind; nothing in it has
+ *   to start at zero (each call rewrites what it later reads).  Calls that overlap on
+ *   the GPU (on different streams, or from different threads) race on the array and
+ *   must be serialised by the caller.
+ */
+#define ATTN_DECODE_NOALLOC_MAX_SCRATCH (32u << 20)
+attn_status attn_decode_paged_noalloc(const void* q, const void* k_pool, const void* v_pool,
+                                      const int32_t* block_table, const int32_t* seq_lens,
+                                      int page_size, void* o, float* lse, int num_seqs, int Hq,
+                                      int Hkv, int d, int num_pages, int max_pages_per_seq,
+                                      float scale, void* stream);
+
+/* Size in bytes of the static scratch of attn_decode_paged_noalloc. */
+size_t attn_decode_paged_noalloc_max_scratch(void);
 
 /*
  * attn_get_device_status — synchronises `stream`, then returns and clears the first
