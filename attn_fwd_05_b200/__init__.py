@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     attn_fwd,
     attn_fwd_ex,
     attn_get_device_status,
+    attn_debug_exp2,
     attn_debug_watchdog,
     attn_status_string,
     library_path,

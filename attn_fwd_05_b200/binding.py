@@ -38,6 +38,7 @@ SIGNATURES = {
                                        _P]),
     "attn_decode_paged_noalloc_max_scratch": (ctypes.c_size_t, []),
     "attn_debug_watchdog": (_I, [ctypes.c_uint64, _P]),
+    "attn_debug_exp2": (_I, [_P, _P, _I, _P]),
     "attn_get_device_status": (_I, [_P]),
     "attn_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -186,6 +187,15 @@ def attn_get_device_status(stream=None) -> int:
 
 def attn_debug_watchdog(timeout_ns: int, stream=None) -> None:
     _check(load_library().attn_debug_watchdog(int(timeout_ns), _stream(stream)), "attn_debug_watchdog")
+
+
+def attn_debug_exp2(x: torch.Tensor, y: torch.Tensor, stream=None) -> None:
+    """y = 2^x by the kernel's FMA-pipe polynomial (fp32 device tensors)."""
+    n = x.numel()
+    if y.numel() != n:
+        raise ValueError("x and y must have the same size")
+    _check(load_library().attn_debug_exp2(_dev(x, "x", torch.float32), _dev(y, "y", torch.float32), n,
+                                          _stream(stream)), "attn_debug_exp2")
 
 
 def attn_status_string(status: int) -> str:

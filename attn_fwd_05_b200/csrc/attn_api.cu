@@ -362,6 +362,15 @@ attn_status attn_debug_watchdog(uint64_t timeout_ns, void* stream) {
   return launch_status();
 }
 
+attn_status attn_debug_exp2(const float* x, float* y, int n, void* stream) {
+  if (n < 0 || (n > 0 && (x == nullptr || y == nullptr))) return ATTN_ERR_INVALID_ARG;
+  if (n == 0) return ATTN_OK;
+  const int threads = 256;
+  const int blocks = (int)(((long long)n + 2 * threads - 1) / (2 * threads));
+  attn::attn_exp2_poly_kernel<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return launch_status();
+}
+
 attn_status attn_get_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
   int v = 0;

@@ -22,10 +22,11 @@
 //     idea for Blackwell).  TMEM: S0 | S1 | O0 | O1 = 128 + 128 + d + d columns.
 //   * Kernel "single" (d = 256): one Q tile, S double-buffered in TMEM (64 + 64 columns)
 //     next to O (256 columns), so the next S = Q K^T runs while the softmax works.
-//   * The rescale of O is skipped unless a row maximum grows by more than 2^8; the
-//     stale maximum stays exact because O and both row sums use the same reference.
-//     O is normalised by the sum of the bf16-rounded P that actually multiplied V, and
-//     the log-sum-exp uses the fp32 sum of the unrounded P.
+//   * The reference of each row is its exact running maximum: whenever a block raises
+//     it, the row's O accumulator is rescaled in TMEM before the next P V.  The row's
+//     largest probability is then exactly 1 and its bf16 rounding is exact, which keeps
+//     sharply peaked rows accurate; O and the log-sum-exp are normalised by the one
+//     fp32 sum of the probabilities.
 #pragma once
 
 #include "sm100_common.cuh"
@@ -33,7 +34,6 @@
 namespace attn {
 
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
 struct FwdArgs {
   CUtensorMap tm_q;  // [B*Hq, Nq, d] bf16, box {64, 128, 1}
@@ -123,63 +123,6 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
   }
 }
 
-// One softmax step for the calling thread's row over NCOL score columns held in TMEM.
-// Writes the bf16 probabilities over the first NCOL/2 columns of the same TMEM block.
-// Returns the factor the row's O accumulator must be multiplied by (1 when the
-// reference maximum did not move).
-template <int NCOL>
-__device__ __forceinline__ float softmax_step(uint32_t s_taddr, bool masked, int col_limit, float sl2,
-                                              float& m, float& l, float& lr) {
-  static_assert(NCOL == 64 || NCOL == 128, "score block width");
-  uint32_t r[NCOL];
-#pragma unroll
-  for (int c = 0; c < NCOL / 32; ++c) tmem_ld32(s_taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
-#pragma unroll
-  for (int c = 0; c < NCOL / 32; ++c) tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
-
-  float s[NCOL];
-#pragma unroll
-  for (int c = 0; c < NCOL; ++c) s[c] = __uint_as_float(r[c]);
-  if (masked) {
-#pragma unroll
-    for (int c = 0; c < NCOL; ++c) s[c] = (c > col_limit) ? -INFINITY : s[c];
-  }
-  float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-  for (int c = 4; c < NCOL; c += 4) {
-    mx0 = fmaxf(mx0, s[c]);
-    mx1 = fmaxf(mx1, s[c + 1]);
-    mx2 = fmaxf(mx2, s[c + 2]);
-    mx3 = fmaxf(mx3, s[c + 3]);
-  }
-  const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-  float alpha = 1.0f;
-  if (mx > m + kRescaleThreshold) {  // false while nothing is visible (mx = -inf)
-    alpha = ex2(m - mx);             // 0 when m = -inf
-    m = mx;
-  }
-  const float mu = (m == -INFINITY) ? 0.0f : m;
-
-  uint32_t P[NCOL / 2];
-  float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-#pragma unroll
-  for (int i = 0; i < NCOL / 2; ++i) {
-    const float p0 = ex2(fmaf(s[2 * i], sl2, -mu));
-    const float p1 = ex2(fmaf(s[2 * i + 1], sl2, -mu));
-    a0 += p0;
-    a1 += p1;
-    const uint32_t w = pack_bf16x2(p0, p1);
-    P[i] = w;
-    b0 += bf16lo_to_f32(w);
-    b1 += bf16hi_to_f32(w);
-  }
-#pragma unroll
-  for (int c = 0; c < NCOL / 64; ++c) tmem_st32(s_taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&P[c * 32]));
-  l = l * alpha + (a0 + a1);
-  lr = lr * alpha + (b0 + b1);
-  return alpha;
-}
-
 // Multiplies the calling thread's O row (D fp32 columns in TMEM) by alpha.
 template <int D>
 __device__ __forceinline__ void rescale_o(uint32_t o_taddr, float alpha) {
@@ -194,11 +137,11 @@ __device__ __forceinline__ void rescale_o(uint32_t o_taddr, float alpha) {
   }
 }
 
-// Epilogue for one row: O / lr to global (bf16 or fp32) and the log-sum-exp.
+// Epilogue for one row: O / l to global (bf16 or fp32) and the log-sum-exp.
 template <int D>
 __device__ __forceinline__ void store_row(const FwdArgs& a, uint32_t o_taddr, bool have_o, bool valid, int b,
-                                          int hq, int q, float m, float l, float lr) {
-  const float inv = lr > 0.f ? 1.0f / lr : 0.f;
+                                          int hq, int q, float m, float l) {
+  const float inv = l > 0.f ? 1.0f / l : 0.f;
   const size_t row = ((size_t)b * a.Hq + hq) * (size_t)a.Nq + (size_t)(valid ? q : 0);
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {
@@ -239,18 +182,32 @@ __device__ __forceinline__ void store_row(const FwdArgs& a, uint32_t o_taddr, bo
 // ====================================================================================
 // Kernel 1: two Q tiles per CTA (d = 64 or 128)
 // ====================================================================================
+//
+// Warp roles (640 threads): warp 0 issues TMA loads, warp 1 issues the MMAs, warps 2-3
+// idle, warps 4-19 are four softmax warpgroups: tile t, column half h handled by
+// warpgroup 1 + 2t + h.  Each softmax thread owns one query row of its tile and 64 of
+// the 128 score columns of a block; the two halves of a row exchange their block
+// maxima through shared memory, so both apply the same reference.  Two warps per
+// scheduler work on a tile's softmax at once, which keeps the exp unit busy while the
+// other warp issues its arithmetic.
+//
+// P is written over the half's own score columns (keys 64h..64h+63 of the block go
+// to TMEM columns 64h..64h+31 of the S block), so neither half can overwrite scores the
+// other still has to read.
 
 template <int D>
 struct PingPongCfg {
   static constexpr int BM = 128;
   static constexpr int BN = 128;
-  static constexpr int THREADS = 384;  // warp 0 TMA, warp 1 MMA, warps 4-7 and 8-11 softmax
+  static constexpr int THREADS = 640;
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int NSTAGE = (D == 64) ? 8 : 4;  // K and V tiles share the ring
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * Q_BYTES;
-  static constexpr int OFF_BAR = OFF_KV + NSTAGE * KV_BYTES;
+  static constexpr int OFF_RED = OFF_KV + NSTAGE * KV_BYTES;  // row-max / row-sum exchange
+  static constexpr int RED_BYTES = 2 * 2 * 2 * 128 * 4 + 2 * 2 * 128 * 4;
+  static constexpr int OFF_BAR = OFF_RED + RED_BYTES;
   static constexpr int SMEM = OFF_BAR + 512 + 1024;  // barriers + 1 KB alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
@@ -260,7 +217,8 @@ struct PingPongBars {
   uint64_t q_full[2];
   uint64_t s_full[2];
   uint64_t p_full[2];
-  uint64_t o_done[2];
+  uint64_t o_done[2];   // one phase per P V of the tile
+  uint64_t o_final[2];  // one phase: the tile's last P V is done
   uint64_t drain;
   uint64_t kv_full[8];
   uint64_t kv_empty[8];
@@ -268,35 +226,206 @@ struct PingPongBars {
   int abort_flag;
 };
 
+// Exchange area: block maxima [tile][block parity][half][row] and final row sums
+// [tile][half][row].
+struct PingPongRed {
+  float xmax[2][2][2][128];
+  float sums[2][2][128];
+};
+
+// P V for one tile: k-step kk covers keys 16kk..16kk+15, whose packed P sits at TMEM
+// column 64*(kk/4) + 8*(kk%4) of the S block (each column half keeps its own P).
+template <int D, int BN>
+__device__ __forceinline__ void issue_pv_split(uint32_t o_tmem, uint32_t s_tmem, uint32_t sV, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk) {
+    const uint64_t db = smem_desc_sw128(sV + kk * (16 * 128), BN * 128, 1024);
+    mma_ts(o_tmem, s_tmem + (kk >> 2) * 64 + (kk & 3) * 8, db, idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Three pairs of probabilities in every eight (kEmuMask) are computed on the FMA pipe
+// (exp2_fma2) instead of the exp unit: per block the exp unit alone would otherwise need
+// as many cycles as the tensor core, the bottleneck the FA4 page names for Blackwell
+// (section "Softmax distribué et émulé").  The split balances the exp unit against the
+// issue slots the polynomial costs.
+constexpr uint32_t kEmuMask = 0xA4u;  // pairs 2, 5 and 7 of each group of 8
+
+// p = 2^(s * sl2 + nmu) for 32 pairs; the packed bf16 values go to TMEM at p_taddr in
+// two 16-column stores (so fewer of them are held in registers), (a0 + a1) gets the
+// fp32 sum.
+template <uint32_t MASK>
+__device__ __forceinline__ void exp_pairs(const float (&s)[64], float sl2, float nmu, uint32_t p_taddr, float& a0,
+                                          float& a1) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint32_t P[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int i = 16 * half + k;
+      float y0, y1, p0, p1;
+      fma2(y0, y1, s[2 * i], s[2 * i + 1], sl2, sl2, nmu, nmu);
+      if ((MASK >> (i & 7)) & 1u) {
+        exp2_fma2(p0, p1, y0, y1);
+      } else {
+        p0 = ex2(y0);
+        p1 = ex2(y1);
+      }
+      add2(a0, a1, p0, p1);
+      P[k] = pack_bf16x2(p0, p1);
+    }
+    tmem_st16(p_taddr + 16 * half, P);
+  }
+}
+
+// Softmax over this thread's 64 columns of one row.  Returns the factor for the row's O.
+//
+// The exchange barrier also ORs `stop` over both halves, so that they leave the block
+// loop at the same block (a half that left alone would hang the other on the barrier).
+__device__ __forceinline__ float softmax_half_step(uint32_t s_taddr, bool masked, int col_limit, float sl2,
+                                                   float* xmax_mine, const float* xmax_other, int bar_id,
+                                                   float& m, float& l, bool& stop) {
+  uint32_t r[64];
+  tmem_ld32(s_taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  tmem_ld32(s_taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+  tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+  float s[64];
+#pragma unroll
+  for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(r[c]);
+  if (masked) {
+#pragma unroll
+    for (int c = 0; c < 64; ++c) s[c] = (c > col_limit) ? -INFINITY : s[c];
+  }
+  float x0 = max3(s[0], s[1], s[2]), x1 = max3(s[3], s[4], s[5]);
+#pragma unroll
+  for (int c = 6; c < 62; c += 4) {
+    x0 = max3(x0, s[c], s[c + 1]);
+    x1 = max3(x1, s[c + 2], s[c + 3]);
+  }
+  float mx = max3(x0, x1, fmaxf(s[62], s[63])) * sl2;
+  *xmax_mine = mx;
+  stop = named_bar_sync_or(bar_id, 256, stop);
+  mx = fmaxf(mx, *xmax_other);
+
+  float alpha = 1.0f;
+  if (mx > m) {            // false while nothing is visible (mx = -inf)
+    alpha = ex2(m - mx);   // 0 when m = -inf
+    m = mx;
+  }
+  const float nmu = (m == -INFINITY) ? 0.0f : -m;
+
+  float a0 = 0.f, a1 = 0.f;
+  if (masked) {
+    exp_pairs<0u>(s, sl2, nmu, s_taddr, a0, a1);  // -inf entries: the exp unit returns exact zeros
+  } else {
+    exp_pairs<kEmuMask>(s, sl2, nmu, s_taddr, a0, a1);
+  }
+  l = l * alpha + (a0 + a1);
+  return alpha;
+}
+
+template <int NC>
+__device__ __forceinline__ void rescale_cols(uint32_t o_taddr, float alpha) {
+#pragma unroll
+  for (int c = 0; c < NC / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(o_taddr + c * 32, r);
+    tmem_ld_wait(r);
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      float u0 = __uint_as_float(r[i]), u1 = __uint_as_float(r[i + 1]);
+      mul2(u0, u1, alpha, alpha);
+      r[i] = __float_as_uint(u0);
+      r[i + 1] = __float_as_uint(u1);
+    }
+    tmem_st32(o_taddr + c * 32, r);
+  }
+}
+
+// Epilogue for NC columns of one row: O / l to global (bf16 or fp32).
+template <int NC>
+__device__ __forceinline__ void store_cols(const FwdArgs& a, uint32_t o_taddr, bool have_o, bool valid,
+                                           size_t elem_off, float l) {
+  const float inv = l > 0.f ? 1.0f / l : 0.f;
+#pragma unroll
+  for (int c = 0; c < NC / 32; ++c) {
+    uint32_t r[32];
+    if (have_o) {
+      tmem_ld32(o_taddr + c * 32, r);
+      tmem_ld_wait(r);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) r[i] = 0u;
+    }
+    if (valid) {
+      if (a.o_f32) {
+        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.o) + elem_off + c * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
+                               __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv);
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + elem_off + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv, __uint_as_float(r[8 * i + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv, __uint_as_float(r[8 * i + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv, __uint_as_float(r[8 * i + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv, __uint_as_float(r[8 * i + 7]) * inv);
+          dst[i] = w;
+        }
+      }
+    }
+  }
+}
+
 template <int D>
-__global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_constant__ FwdArgs a) {
+__global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_constant__ FwdArgs a) {
   using C = PingPongCfg<D>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   PingPongBars* bars = reinterpret_cast<PingPongBars*>(smem + C::OFF_BAR);
+  PingPongRed* red = reinterpret_cast<PingPongRed*>(smem + C::OFF_RED);
   volatile int* abort_flag = &bars->abort_flag;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit (heaviest causal tiles first)
+  // ---- work unit.  Causal: heaviest q-tiles first (longest-processing-time order).
+  // Non-causal: all units weigh the same; consecutive CTAs share a head so that the
+  // K/V tiles they all stream stay in L2.
   int b, kvh;
   TileJob tj[2];
   {
     const int u = blockIdx.x;
     if (a.pair_heads) {
-      const int per_level = a.B * (a.Hq / 2);
-      const int qt = a.n_qtiles - 1 - u / per_level;
-      const int rem = u % per_level;
-      b = rem / (a.Hq / 2);
-      const int h0 = 2 * (rem % (a.Hq / 2));
+      const int hp_n = a.Hq / 2;
+      int qt, rem;
+      if (a.causal) {
+        qt = a.n_qtiles - 1 - u / (a.B * hp_n);
+        rem = u % (a.B * hp_n);
+      } else {
+        qt = u % a.n_qtiles;
+        rem = u / a.n_qtiles;
+      }
+      b = rem / hp_n;
+      const int h0 = 2 * (rem % hp_n);
       tj[0] = make_tile<BN>(a, h0, qt * 128);
       tj[1] = make_tile<BN>(a, h0 + 1, qt * 128);
     } else {
-      const int per_level = a.B * a.Hq;
-      const int qp = (a.n_qtiles + 1) / 2 - 1 - u / per_level;
-      const int rem = u % per_level;
+      const int nqp = (a.n_qtiles + 1) / 2;
+      int qp, rem;
+      if (a.causal) {
+        qp = nqp - 1 - u / (a.B * a.Hq);
+        rem = u % (a.B * a.Hq);
+      } else {
+        qp = u % nqp;
+        rem = u / nqp;
+      }
       b = rem / a.Hq;
       const int h = rem % a.Hq;
       tj[0] = make_tile<BN>(a, h, (2 * qp) * 128);
@@ -310,8 +439,9 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->q_full[t], 1);
       mbar_init(&bars->s_full[t], 1);
-      mbar_init(&bars->p_full[t], 4);
+      mbar_init(&bars->p_full[t], 8);
       mbar_init(&bars->o_done[t], 1);
+      mbar_init(&bars->o_final[t], 1);
     }
     mbar_init(&bars->drain, 1);
     for (int s = 0; s < C::NSTAGE; ++s) {
@@ -374,14 +504,17 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
       }
     }
   } else if (warp == 1) {
-    // ================= MMA issuer
+    // ================= MMA issuer.  Order per block j:
+    //   PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)
+    // so one tile's softmax overlaps the other tile's two MMAs.  S_t(j+1) overwrites
+    // the TMEM block that held P_t(j); it is issued after PV_t(j), and the tensor core
+    // executes one thread's MMAs in issue order.
     if (lane == 0 && nblk > 0) {
       bool ok = true;
       for (int t = 0; t < 2 && ok; ++t)
         if (tj[t].nblk > 0) ok = mbar_wait(&bars->q_full[t], 0, abort_flag, a.timeout_ns);
       auto stage_of = [&](int it) { return it % C::NSTAGE; };
       auto parity_of = [&](int it) { return (uint32_t)((it / C::NSTAGE) & 1); };
-      // prologue: S_t(0)
       if (ok) ok = mbar_wait(&bars->kv_full[stage_of(0)], parity_of(0), abort_flag, a.timeout_ns);
       if (ok) {
         tc_fence_after();
@@ -407,8 +540,9 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
               break;
             }
             tc_fence_after();
-            issue_pv<D, BN>(tmem + colO, tmem + colS, sV, j > 0);
+            issue_pv_split<D, BN>(tmem + colO, tmem + colS, sV, j > 0);
             tc_commit(&bars->o_done[t]);
+            if (j + 1 == tj[t].nblk) tc_commit(&bars->o_final[t]);
           }
           if (t == 1) tc_commit(&bars->kv_empty[stage_of(itV)]);
           if (next && j + 1 < tj[t].nblk) {
@@ -437,46 +571,65 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
       mbar_wait(&bars->drain, 0, abort_flag, a.timeout_ns, false);
     }
   } else if (warp >= 4) {
-    // ================= softmax warpgroups: warps 4-7 own tile 0, warps 8-11 tile 1
-    const int t = (warp - 4) >> 2;
-    const int quad = warp & 3;            // TMEM lane quadrant this warp may access
-    const int r = quad * 32 + lane;       // row within the tile
+    // ================= softmax: warpgroup 1 + 2t + h owns tile t, column half h
+    const int sw = warp - 4;
+    const int t = sw >> 3;
+    const int h = (sw >> 2) & 1;
+    const int quad = warp & 3;       // TMEM lane quadrant this warp may access
+    const int r = quad * 32 + lane;  // row within the tile
     const TileJob& job = tj[t];
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t s_addr = tmem + lane_off + (t ? C::COL_S1 : C::COL_S0);
-    const uint32_t o_addr = tmem + lane_off + (t ? C::COL_O1 : C::COL_O0);
+    const uint32_t s_addr = tmem + lane_off + (t ? C::COL_S1 : C::COL_S0) + 64 * h;
+    const uint32_t o_addr = tmem + lane_off + (t ? C::COL_O1 : C::COL_O0) + (D / 2) * h;
     const int q = job.q0 + r;
-    const int klim = row_key_limit(a, q);
-    float m = -INFINITY, l = 0.f, lr = 0.f;
+    const int klim = row_key_limit(a, q) - 64 * h;  // limit relative to this half's first column
+    const int bar_id = 1 + t;
+    float m = -INFINITY, l = 0.f;
     bool ok = true;
+    bool fail = false;  // a wait of this warp gave up; decided jointly at the next exchange
     for (int j = 0; j < job.nblk; ++j) {
-      if (!mbar_wait(&bars->s_full[t], j & 1, abort_flag, a.timeout_ns)) {
-        ok = false;
-        break;
-      }
+      // both halves reach the exchange barrier of every block; an abort is decided
+      // jointly there
+      bool stop = fail || !mbar_wait(&bars->s_full[t], j & 1, abort_flag, a.timeout_ns) || *abort_flag;
       tc_fence_after();
       const bool masked = block_needs_mask<BN>(a, job, j);
-      const float alpha = softmax_step<BN>(s_addr, masked, klim - j * BN, a.scale_log2, m, l, lr);
+      const float alpha = softmax_half_step(s_addr, masked, klim - j * BN, a.scale_log2,
+                                            &red->xmax[t][j & 1][h][r], &red->xmax[t][j & 1][h ^ 1][r], bar_id,
+                                            m, l, stop);
+      if (stop) {
+        fail = true;
+        break;
+      }
       if (__any_sync(0xffffffffu, alpha != 1.0f) && j > 0) {
         // O holds P V of blocks < j: wait for the last of those MMAs, then rescale
-        if (!mbar_wait(&bars->o_done[t], (j - 1) & 1, abort_flag, a.timeout_ns)) {
-          ok = false;
-          break;
+        if (mbar_wait(&bars->o_done[t], (j - 1) & 1, abort_flag, a.timeout_ns)) {
+          tc_fence_after();
+          rescale_cols<D / 2>(o_addr, alpha);
+        } else {
+          fail = true;
         }
-        tc_fence_after();
-        rescale_o<D>(o_addr, alpha);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full[t]);
     }
-    bool have_o = job.nblk > 0;
+    ok = !fail;
+    const bool have_o = job.nblk > 0;
     if (ok && have_o) {
-      ok = mbar_wait(&bars->o_done[t], (job.nblk - 1) & 1, abort_flag, a.timeout_ns);
+      ok = mbar_wait(&bars->o_final[t], 0, abort_flag, a.timeout_ns);
       tc_fence_after();
     }
-    if (ok) store_row<D>(a, o_addr, have_o, r < job.rows, b, job.hq, q, m, l, lr);
+    // combine the two halves' row sums (same reference maximum, same rescale history)
+    red->sums[t][h][r] = l;
+    named_bar_sync(bar_id, 256);
+    l += red->sums[t][h ^ 1][r];
+    if (ok) {
+      const bool valid = r < job.rows;
+      const size_t row = ((size_t)b * a.Hq + job.hq) * (size_t)a.Nq + (size_t)(valid ? q : 0);
+      store_cols<D / 2>(a, o_addr, have_o, valid, row * D + (D / 2) * h, l);
+      if (h == 0 && valid && a.lse != nullptr) a.lse[row] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
+    }
   }
 
   tc_fence_before();
@@ -490,6 +643,45 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
 // ====================================================================================
 // Kernel 2: one Q tile per CTA, S double-buffered (d = 256)
 // ====================================================================================
+
+// Softmax over the calling thread's whole 64-column row of one score block (one
+// warpgroup per tile).  Returns the factor for the row's O.
+__device__ __forceinline__ float softmax_row64_step(uint32_t s_taddr, bool masked, int col_limit, float sl2,
+                                                    float& m, float& l) {
+  uint32_t r[64];
+  tmem_ld32(s_taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  tmem_ld32(s_taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+  tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+  float s[64];
+#pragma unroll
+  for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(r[c]);
+  if (masked) {
+#pragma unroll
+    for (int c = 0; c < 64; ++c) s[c] = (c > col_limit) ? -INFINITY : s[c];
+  }
+  float x0 = max3(s[0], s[1], s[2]), x1 = max3(s[3], s[4], s[5]);
+#pragma unroll
+  for (int c = 6; c < 62; c += 4) {
+    x0 = max3(x0, s[c], s[c + 1]);
+    x1 = max3(x1, s[c + 2], s[c + 3]);
+  }
+  const float mx = max3(x0, x1, fmaxf(s[62], s[63])) * sl2;
+  float alpha = 1.0f;
+  if (mx > m) {
+    alpha = ex2(m - mx);
+    m = mx;
+  }
+  const float nmu = (m == -INFINITY) ? 0.0f : -m;
+  float a0 = 0.f, a1 = 0.f;
+  if (masked) {
+    exp_pairs<0u>(s, sl2, nmu, s_taddr, a0, a1);
+  } else {
+    exp_pairs<kEmuMask>(s, sl2, nmu, s_taddr, a0, a1);
+  }
+  l = l * alpha + (a0 + a1);
+  return alpha;
+}
 
 template <int D>
 struct SingleCfg {
@@ -511,7 +703,8 @@ struct SingleBars {
   uint64_t q_full;
   uint64_t s_full[2];
   uint64_t p_full[2];
-  uint64_t o_done;
+  uint64_t o_done;   // one phase per P V
+  uint64_t o_final;  // one phase: the last P V is done
   uint64_t drain;
   uint64_t kv_full[8];
   uint64_t kv_empty[8];
@@ -535,8 +728,8 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
   {
     const int u = blockIdx.x;
     const int per_level = a.B * a.Hq;
-    const int qt = a.n_qtiles - 1 - u / per_level;
-    const int rem = u % per_level;
+    const int qt = a.causal ? a.n_qtiles - 1 - u / per_level : u % a.n_qtiles;
+    const int rem = a.causal ? u % per_level : u / a.n_qtiles;
     b = rem / a.Hq;
     hq = rem % a.Hq;
     job = make_tile<BN>(a, hq, qt * 128);
@@ -551,6 +744,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
       mbar_init(&bars->p_full[i], 4);
     }
     mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->o_final, 1);
     mbar_init(&bars->drain, 1);
     for (int s = 0; s < C::NSTAGE; ++s) {
       mbar_init(&bars->kv_full[s], 1);
@@ -629,6 +823,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
         tc_fence_after();
         issue_pv<D, BN>(tmem + C::COL_O, tmem + colS(j), sKV + stage_of(itV) * C::KV_BYTES, j > 0);
         tc_commit(&bars->o_done);
+        if (j + 1 == nblk) tc_commit(&bars->o_final);
         tc_commit(&bars->kv_empty[stage_of(itV)]);
         if (j + 2 < nblk) {
           const int itK = 2 * (j + 2);
@@ -649,7 +844,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
     const uint32_t o_addr = tmem + lane_off + C::COL_O;
     const int q = job.q0 + r;
     const int klim = row_key_limit(a, q);
-    float m = -INFINITY, l = 0.f, lr = 0.f;
+    float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nblk; ++j) {
       if (!mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag, a.timeout_ns)) {
@@ -659,8 +854,10 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
       tc_fence_after();
       const uint32_t s_addr = tmem + lane_off + ((j & 1) ? C::COL_S1 : C::COL_S0);
       const bool masked = block_needs_mask<BN>(a, job, j);
-      const float alpha = softmax_step<BN>(s_addr, masked, klim - j * BN, a.scale_log2, m, l, lr);
+      const float alpha = softmax_row64_step(s_addr, masked, klim - j * BN, a.scale_log2, m, l);
       if (__any_sync(0xffffffffu, alpha != 1.0f) && j > 0) {
+        // P V(j-2) finished before S(j) (issued after it), so o_done is in phase j-1 or
+        // later and its parity names P V(j-1) without ambiguity
         if (!mbar_wait(&bars->o_done, (j - 1) & 1, abort_flag, a.timeout_ns)) {
           ok = false;
           break;
@@ -675,10 +872,12 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
     }
     const bool have_o = nblk > 0;
     if (ok && have_o) {
-      ok = mbar_wait(&bars->o_done, (nblk - 1) & 1, abort_flag, a.timeout_ns);
+      // o_final, not o_done: the next Q K^T runs ahead of P V here, so P V(nblk-2) may
+      // still be in flight and o_done's parity could name an older completed phase
+      ok = mbar_wait(&bars->o_final, 0, abort_flag, a.timeout_ns);
       tc_fence_after();
     }
-    if (ok) store_row<D>(a, o_addr, have_o, r < job.rows, b, hq, q, m, l, lr);
+    if (ok) store_row<D>(a, o_addr, have_o, r < job.rows, b, hq, q, m, l);
   }
 
   tc_fence_before();

@@ -249,6 +249,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------------ arithmetic
@@ -257,6 +266,82 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed fp32 pairs (sm_100): one instruction does two lanes of work.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                     float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {  // d += a
+  asm("{\n\t.reg .b64 ra, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rd, {%0, %1};\n\t"
+      "add.rn.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1));
+}
+
+__device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1) {  // d *= a
+  asm("{\n\t.reg .b64 ra, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rd, {%0, %1};\n\t"
+      "mul.rn.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1));
+}
+
+// 2^x for two lanes on the FMA pipe, for x up to 2^22 (inputs below -125 are clamped
+// to -125).  Cody and Waite's reduction x = n + f, n = round(x) (adding 1.5 * 2^23 rounds
+// to an integer), f in [-1/2, 1/2]; 2^f from a degree-3 polynomial fitted by a Remez
+// exchange for minimum relative error (fit_exp2_poly.py; max relative error 7.5e-5);
+// 2^n is added to the exponent field.  Relative error stays below 1e-4.
+constexpr float kExp2C0 = 0x1.fff692p-1f;
+constexpr float kExp2C1 = 0x1.62f31ap-1f;
+constexpr float kExp2C2 = 0x1.f0de1ap-3f;
+constexpr float kExp2C3 = 0x1.c3f76p-5f;
+
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                     float c1);
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1);
+
+__device__ __forceinline__ void exp2_fma2(float& y0, float& y1, float x0, float x1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  float t0 = x0, t1 = x1;
+  add2(t0, t1, kRound, kRound);  // round to nearest integer, kept in the low mantissa bits
+  float n0 = t0, n1 = t1;
+  add2(n0, n1, -kRound, -kRound);  // n = round(x), exact
+  float f0, f1;
+  fma2(f0, f1, n0, n1, -1.0f, -1.0f, x0, x1);  // f = x - n
+  float p0, p1;
+  fma2(p0, p1, f0, f1, kExp2C3, kExp2C3, kExp2C2, kExp2C2);
+  fma2(p0, p1, p0, p1, f0, f1, kExp2C1, kExp2C1);
+  fma2(p0, p1, p0, p1, f0, f1, kExp2C0, kExp2C0);
+  // the low 9 bits of t's encoding hold n (two's complement): shift them into the exponent
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// Evaluates exp2_fma2 over an array (used by the tests of the polynomial).
+__global__ void attn_exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    exp2_fma2(y[i], y[i + 1], x[i], x[i + 1]);
+  } else if (i < n) {
+    float d;
+    exp2_fma2(y[i], d, x[i], 0.0f);
+  }
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -59,6 +59,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="bounded CPU-baseline sample length")
+    p.add_argument("--decode-seqs", type=int, default=64,
+                   help="sequences in the decode batch (64 is the workload; fewer only for small profiles)")
     return p.parse_args()
 
 
@@ -179,9 +181,11 @@ def make_prefill(shape, seed, dev):
     return {"host": (q, k, v), "dev": (q.to(dev), k.to(dev), v.to(dev)), "o": o, "lse": lse}
 
 
-def make_decode(seed, dev):
+def make_decode(seed, dev, nseqs=64):
+    import dataclasses
+
     import attn_fwd_05_b200 as ab
-    s = synth.WORKLOADS["paged_decode_gqa"]
+    s = dataclasses.replace(synth.WORKLOADS["paged_decode_gqa"], S=nseqs)
     kv = synth.decode_inputs(s, seed)
     S = s.S
     ws_bytes = ab.attn_decode_paged_workspace_size(S, s.Hq, s.Hkv, s.d, kv.max_pages_per_seq, s.page_size)
@@ -285,7 +289,7 @@ def config_block(args, shape):
                        "causal": shape.causal, "qk_std": shape.qk_std}}
     if args.workload == "serving_step":
         s = synth.WORKLOADS["paged_decode_gqa"]
-        cfg["decode"] = {"seqs": s.S, "Hq": s.Hq, "Hkv": s.Hkv, "d": s.d, "page_size": s.page_size,
+        cfg["decode"] = {"seqs": args.decode_seqs, "Hq": s.Hq, "Hkv": s.Hkv, "d": s.d, "page_size": s.page_size,
                          "len_range": [s.len_lo, s.len_hi]}
         cfg["l2"] = "inputs larger than L2: each step's 4.6 GB decode KV stream evicts the prefill inputs"
     else:
@@ -303,7 +307,7 @@ def run_ours(args, dist):
     shape = prefill_shape(args.workload)
     seed = synth.workload_seed("gqa_causal_2k" if args.workload == "serving_step" else args.workload)
     pre = make_prefill(shape, seed + 7919 * dist.rank, dev)
-    dec = make_decode(synth.workload_seed("paged_decode_gqa") + 7919 * dist.rank, dev) \
+    dec = make_decode(synth.workload_seed("paged_decode_gqa") + 7919 * dist.rank, dev, args.decode_seqs) \
         if args.workload == "serving_step" else None
     flush = None if dec is not None else torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     scale = synth.default_scale(shape.d)

@@ -193,6 +193,14 @@ attn_status attn_get_device_status(void* stream);
  */
 attn_status attn_debug_watchdog(uint64_t timeout_ns, void* stream);
 
+/*
+ * attn_debug_exp2 — evaluates, for i < n, y[i] = 2^x[i] with the polynomial exponential
+ * the prefill kernel runs on the FMA pipe for part of its probabilities (range
+ * reduction x = n + f, degree-3 minimax polynomial for 2^f).  x and y are device fp32
+ * arrays of n elements; inputs below -125 are clamped to -125.  For testing.
+ */
+attn_status attn_debug_exp2(const float* x, float* y, int n, void* stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* attn_status_string(int status);
 
