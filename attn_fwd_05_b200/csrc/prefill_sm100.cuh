@@ -102,13 +102,19 @@ __device__ __forceinline__ int row_key_limit(const FwdArgs& a, int q) {
   return (int)lim;
 }
 
+// The MMA-issuing thread shares its scheduler with four busy softmax warps, so every
+// instruction it needs per MMA costs it dearly: descriptors are built once and each
+// k-step only adds its byte offset / 16 to the start-address field (offsets stay
+// inside one tile, so the 14-bit field never carries).
 template <int D, int BN>
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t sQ, uint32_t sK) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, BN, 0, 0);
+  const uint64_t da0 = smem_desc_sw128(sQ, 16, 1024);
+  const uint64_t db0 = smem_desc_sw128(sK, 16, 1024);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint64_t da = smem_desc_sw128(sQ + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
-    const uint64_t db = smem_desc_sw128(sK + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024);
+    const uint64_t da = da0 + (uint64_t)((((kk >> 2) * (128 * 128) + (kk & 3) * 32)) >> 4);
+    const uint64_t db = db0 + (uint64_t)((((kk >> 2) * (BN * 128) + (kk & 3) * 32)) >> 4);
     mma_ss(s_tmem, da, db, idesc, kk > 0 ? 1u : 0u);
   }
 }
@@ -116,9 +122,10 @@ __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t sQ, uint32_t 
 template <int D, int BN>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t sV, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+  const uint64_t db0 = smem_desc_sw128(sV, BN * 128, 1024);
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk) {
-    const uint64_t db = smem_desc_sw128(sV + kk * (16 * 128), BN * 128, 1024);
+    const uint64_t db = db0 + (uint64_t)((kk * (16 * 128)) >> 4);
     mma_ts(o_tmem, p_tmem + kk * 8, db, idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
@@ -238,9 +245,10 @@ struct PingPongRed {
 template <int D, int BN>
 __device__ __forceinline__ void issue_pv_split(uint32_t o_tmem, uint32_t s_tmem, uint32_t sV, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+  const uint64_t db0 = smem_desc_sw128(sV, BN * 128, 1024);
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk) {
-    const uint64_t db = smem_desc_sw128(sV + kk * (16 * 128), BN * 128, 1024);
+    const uint64_t db = db0 + (uint64_t)((kk * (16 * 128)) >> 4);
     mma_ts(o_tmem, s_tmem + (kk >> 2) * 64 + (kk & 3) * 8, db, idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
@@ -250,7 +258,7 @@ __device__ __forceinline__ void issue_pv_split(uint32_t o_tmem, uint32_t s_tmem,
 // as many cycles as the tensor core, the bottleneck the FA4 page names for Blackwell
 // (section "Softmax distribué et émulé").  The split balances the exp unit against the
 // issue slots the polynomial costs.
-constexpr uint32_t kEmuMask = 0xA4u;  // pairs 2, 5 and 7 of each group of 8
+constexpr uint32_t kEmuMask = 0x00u;  // measured: FMA-pipe exps starve the MMA-issuing warp (see below)
 
 // p = 2^(s * sl2 + nmu) for 32 pairs; the packed bf16 values go to TMEM at p_taddr in
 // two 16-column stores (so fewer of them are held in registers), (a0 + a1) gets the
