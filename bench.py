@@ -51,7 +51,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="serving_step",
@@ -62,6 +62,35 @@ def parse():
     p.add_argument("--decode-seqs", type=int, default=64,
                    help="sequences in the decode batch (64 is the workload; fewer only for small profiles)")
     return p.parse_args()
+
+
+CSRC = ("attn_api.cu", "decode_sm100.cuh", "prefill_sm100.cuh", "sm100_common.cuh")
+
+
+def csrc_digest() -> str:
+    """sha256 prefix of the kernel sources, to match against the committed ncu summaries."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in CSRC:
+        with open(os.path.join(ROOT, "attn_fwd_05_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(profile: str, scale: float = 1.0):
+    """DRAM bytes per launch from a committed ncu summary, or None when the kernel sources
+    changed since it was captured (its counters no longer describe this build)."""
+    path = os.path.join(ROOT, "profiles", profile)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    import re
+    m_sha = re.search(r"csrc sha256 prefix `([0-9a-f]+)`", text)
+    m_b = re.search(r"traffic_bytes_per_launch: (\d+)", text)
+    if not (m_sha and m_b) or m_sha.group(1) != csrc_digest():
+        return None
+    return int(m_b.group(1)) * scale
 
 
 def load_peaks():
@@ -83,6 +112,7 @@ class Dist:
         self.on = self.world > 1
 
     def init(self, backend="nccl"):
+        self.backend = backend
         if self.on:
             import torch.distributed as dist
             dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300),
@@ -94,10 +124,12 @@ class Dist:
             dist.barrier()
 
     def max(self, x: float) -> float:
+        """The maximum of x over all ranks (timings are reported as the slowest rank's)."""
         if not self.on:
             return x
         import torch.distributed as dist
-        t = torch.tensor([x], dtype=torch.float64, device=torch.device("cuda", self.local))
+        dev = torch.device("cuda", self.local) if getattr(self, "backend", "nccl") == "nccl" else torch.device("cpu")
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
@@ -169,6 +201,11 @@ def _num(s):
 
 
 # ----------------------------------------------------------------------------- workloads
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws an independent problem of the same shape (weak scaling)."""
+    return base + 7919 * rank
+
 
 def prefill_shape(name: str):
     return synth.WORKLOADS["gqa_causal_2k" if name == "serving_step" else name]
@@ -306,8 +343,8 @@ def run_ours(args, dist):
     peaks, peak_src = load_peaks()
     shape = prefill_shape(args.workload)
     seed = synth.workload_seed("gqa_causal_2k" if args.workload == "serving_step" else args.workload)
-    pre = make_prefill(shape, seed + 7919 * dist.rank, dev)
-    dec = make_decode(synth.workload_seed("paged_decode_gqa") + 7919 * dist.rank, dev, args.decode_seqs) \
+    pre = make_prefill(shape, rank_seed(seed, dist.rank), dev)
+    dec = make_decode(rank_seed(synth.workload_seed("paged_decode_gqa"), dist.rank), dev, args.decode_seqs) \
         if args.workload == "serving_step" else None
     flush = None if dec is not None else torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     scale = synth.default_scale(shape.d)
@@ -371,6 +408,15 @@ def run_ours(args, dist):
     prefill_tflops = N * flops * K / (pre_sum * 1e-3) / 1e12
     avg_pre_ms = sum(pre_ms) / K
     achieved = flops / (avg_pre_ms * 1e-3) / 1e12
+    kname = "attn_fwd_pingpong_kernel<128>" if shape.d <= 128 else "attn_fwd_single_kernel<256>"
+    prefill_roofline = {
+        "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+        "frac": achieved / peaks["bf16_tflops"],
+        "traffic": profiled_traffic("attn_fwd_pingpong_gqa_causal_2k.md")
+        if args.workload in ("serving_step", "gqa_causal_2k") else None,
+        "peak_source": f"{peak_src} bf16_tflops (burst cuBLAS); frac of the sustained figure "
+                       f"{achieved / peaks['bf16_tflops_sustained']:.3f}",
+        "kernel": kname, "flops_per_launch": flops, "median_ms": statistics.median(pre_ms)}
     line = {
         "metric": METRIC,
         "value": prefill_tflops,
@@ -385,12 +431,7 @@ def run_ours(args, dist):
         "dtype": "bf16",
         "data": "synthetic",
         "config": config_block(args, shape),
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved / peaks["bf16_tflops"], "traffic": None,
-                     "peak_source": f"{peak_src} bf16_tflops (burst cuBLAS); "
-                                    f"frac of sustained {achieved / peaks['bf16_tflops_sustained']:.3f}",
-                     "kernel": "attn_fwd_pingpong_kernel<128>" if shape.d <= 128 else "attn_fwd_single_kernel<256>",
-                     "median_ms": statistics.median(pre_ms)},
+        "roofline": prefill_roofline,
         "gpu_launches": K * (1 + (3 if dec is not None else 0)),
         "clocks": clk,
     }
@@ -398,14 +439,22 @@ def run_ours(args, dist):
         kvb = dec["kv_bytes"]
         avg_dec_ms = sum(dec_ms) / K
         gbs = kvb / (avg_dec_ms * 1e-3) / 1e9
+        full = args.decode_seqs == 64
+        decode_roofline = {
+            "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": gbs / peaks["hbm_gbs"],
+            "traffic": profiled_traffic("attn_decode_split_paged_decode.md") if full else None,
+            "peak_source": f"{peak_src} hbm_gbs (copy)",
+            "kernel": "attn_decode_split_kernel<128> (timed with its plan and merge kernels: one decode call)",
+            "bytes_per_launch": kvb, "median_ms": statistics.median(dec_ms)}
         line["decode"] = {
             "metric": "paged decode KV-read GB/s", "value": N * kvb * K / (dec_sum * 1e-3) / 1e9, "unit": "GB/s",
-            "kv_bytes_per_step": kvb, "median_ms": statistics.median(dec_ms),
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm_gbs"], "traffic": None,
-                         "peak_source": f"{peak_src} hbm_gbs (copy)",
-                         "kernels": "attn_decode_plan + attn_decode_split_kernel<128> + attn_decode_merge_kernel<128>"},
+            "kv_bytes_per_step": kvb, "roofline": decode_roofline,
         }
+        # the decode call takes about 4/5 of the step: it is the step's dominant kernel
+        if avg_dec_ms > avg_pre_ms:
+            line["roofline"] = decode_roofline
+            line["prefill_roofline"] = prefill_roofline
 
     if not args.no_e2e:
         line["e2e"] = e2e_prefill(args, ab, pre, shape, scale, flops, dev, stream, dist)
