@@ -124,7 +124,8 @@ attn_status launch_decode(attn::DecArgs& a, cudaStream_t st, long long max_items
   auto ks = attn::attn_decode_split_kernel<D>;
   const int slot = D == 64 ? 3 : (D == 128 ? 4 : 5);
   if (!ensure_smem(ks, C::SMEM, slot)) return ATTN_ERR_CUDA;
-  attn::attn_decode_plan_kernel<<<1, 1024, 0, st>>>(a.seq_lens, a.S, a.max_pages * a.page_size, a.chunk_prefix);
+  attn::attn_decode_plan_kernel<<<1, 1024, 0, st>>>(a.seq_lens, a.S, a.max_pages * a.page_size, a.chunk_prefix,
+                                                    a.item_map);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   long long grid = (long long)sm_count() * C::CTAS_PER_SM;
   if (grid > max_items) grid = max_items;
@@ -138,7 +139,7 @@ attn_status launch_decode(attn::DecArgs& a, cudaStream_t st, long long max_items
 }
 
 struct DecodeLayout {
-  size_t off_prefix, off_part_o, off_part_lse, total;
+  size_t off_prefix, off_item_map, off_part_o, off_part_lse, total;
   int max_chunks;
 };
 
@@ -151,7 +152,8 @@ bool decode_layout(int S, int Hq, int d, int max_pages, int page_size, DecodeLay
   L->max_chunks = (int)((max_tokens + attn::kDecChunkTok - 1) / attn::kDecChunkTok);
   const size_t parts = (size_t)S * L->max_chunks * Hq;
   L->off_prefix = 0;
-  L->off_part_o = align256((size_t)(S + 1) * 4);
+  L->off_item_map = align256((size_t)(S + 1) * 4);
+  L->off_part_o = L->off_item_map + align256((size_t)S * L->max_chunks * 16);
   L->off_part_lse = L->off_part_o + align256(parts * d * 4);
   L->total = L->off_part_lse + align256(parts * 4);
   return true;
@@ -313,6 +315,7 @@ attn_status attn_decode_paged(const void* q, const void* k_pool, const void* v_p
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.chunk_prefix = reinterpret_cast<int*>(ws + L.off_prefix);
+  a.item_map = reinterpret_cast<int4*>(ws + L.off_item_map);
   a.part_o = reinterpret_cast<float*>(ws + L.off_part_o);
   a.part_lse = reinterpret_cast<float*>(ws + L.off_part_lse);
   a.S = num_seqs;

@@ -110,11 +110,12 @@ def test_decode_empty_batch_is_a_noop(lib):
 
 def test_workspace_size(lib):
     f = lib.attn_decode_paged_workspace_size
-    # 64 sequences, 64 query heads, d = 128, up to 2048 pages of 16 tokens: 32 chunks of 1024 tokens
+    # 64 sequences, 64 query heads, d = 128, up to 2048 pages of 16 tokens: 16 chunks of 2048 tokens
     n = f(64, 64, 8, 128, 2048, 16)
-    parts = 64 * 32 * 64
-    assert n >= parts * 128 * 4 + parts * 4 + 65 * 4
-    assert n < parts * 129 * 4 + 4096
+    parts = 64 * 16 * 64
+    item_map = 64 * 16 * 16  # one 16-byte record per chunk
+    assert n >= parts * 128 * 4 + parts * 4 + 65 * 4 + item_map
+    assert n < parts * 129 * 4 + item_map + 4096
     assert f(64, 64, 8, 96, 2048, 16) == 0    # unsupported head dimension
     assert f(64, 60, 8, 128, 2048, 16) == 0   # Hq not a multiple of Hkv
     assert f(64, 64, 8, 128, 2048, 24) == 0   # unsupported page size

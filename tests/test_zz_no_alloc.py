@@ -67,10 +67,10 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_device):
     lib = binding.load_library()
     limit = lib.attn_decode_paged_noalloc_max_scratch()
     assert limit == 32 << 20
-    # 64 sequences x 64 query heads x d=128 with up to 2048 pages of 16 tokens needs ~68 MB
-    need = lib.attn_decode_paged_workspace_size(64, 64, 8, 128, 2048, 16)
+    # 128 sequences x 64 query heads x d=128 with up to 2048 pages of 16 tokens needs ~68 MB
+    need = lib.attn_decode_paged_workspace_size(128, 64, 8, 128, 2048, 16)
     assert need > limit
     fake = 0x10000
-    st = lib.attn_decode_paged_noalloc(fake, fake, fake, fake, fake, 16, fake, None, 64, 64, 8, 128, 1000, 2048,
+    st = lib.attn_decode_paged_noalloc(fake, fake, fake, fake, fake, 16, fake, None, 128, 64, 8, 128, 1000, 2048,
                                        ctypes.c_float(0.1), None)
     assert st == 8 and lib.attn_status_string(st) == b"ATTN_ERR_TOO_LARGE"
