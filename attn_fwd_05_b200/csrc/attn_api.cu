@@ -150,7 +150,7 @@ bool decode_layout(int S, int Hq, int d, int max_pages, int page_size, DecodeLay
   const long long max_tokens = (long long)max_pages * page_size;
   if (max_tokens > 0x7fffffffLL) return false;
   L->max_chunks = (int)((max_tokens + attn::kDecChunkTok - 1) / attn::kDecChunkTok);
-  const size_t parts = (size_t)S * L->max_chunks * Hq;
+  const size_t parts = (size_t)S * L->max_chunks * attn::kDecWarps * Hq;
   L->off_prefix = 0;
   L->off_item_map = align256((size_t)(S + 1) * 4);
   L->off_part_o = L->off_item_map + align256((size_t)S * L->max_chunks * 16);

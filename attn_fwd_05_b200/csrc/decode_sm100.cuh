@@ -15,14 +15,15 @@
 //     the block table and gathers 16-token pieces of K and V pages with TMA (128-byte
 //     swizzled, 16-byte aligned bulk transfers) into a ring of shared-memory stages; the
 //     next item's pieces are fetched while the current one is still being consumed.
-//     Four consumer warps each own every fourth piece and keep their own online-softmax
-//     state.  All query heads of a KV group share one K/V read ("pack-GQA"): they form
+//     Four consumer warps each own every fourth piece (and their own ring stages) and
+//     keep their own online-softmax state.  All query heads of a KV group share one K/V read ("pack-GQA"): they form
 //     the 16 rows of a warp-level bf16 MMA (m16n8k16), for Q K^T and for P V.  The work
 //     is too small for the tcgen05 path to pay (M would be 8 query heads); the tensor
 //     pipe only has to keep up with HBM here.
-//     At the end of an item the four warp states are merged in shared memory and one
-//     partial (O normalised by its own sum, plus its log2-sum-exp) is written to the
-//     workspace.
+//     At the end of an item each warp writes its state as one partial (O normalised by
+//     its own sum, plus its log2-sum-exp) to the workspace; the warps never wait for one
+//     another (measured: a shared-memory merge of the four states at every item cost
+//     about a tenth of the bandwidth).
 //   * merge kernel: per (sequence, query head) the partials are combined with weights
 //     exp(lse_c - lse), which is exact because the running max/sum statistics of the
 //     online softmax compose associatively.
@@ -117,8 +118,7 @@ struct DecCfg {
   static constexpr int STAGE_BYTES = 2 * PIECE_BYTES;
   static constexpr int NST = (D == 256) ? 4 : 8;        // multiple of kDecWarps
   static constexpr int OFF_RING = 0;
-  static constexpr int OFF_OACC = NST * STAGE_BYTES;              // [16][D] fp32 merge buffer
-  static constexpr int OFF_MISC = OFF_OACC + 16 * D * 4;
+  static constexpr int OFF_MISC = NST * STAGE_BYTES;
   static constexpr int SMEM = OFF_MISC + 1024 + 1024;
   static constexpr int CTAS_PER_SM = (D == 256) ? 2 : 3;
 };
@@ -127,8 +127,6 @@ struct DecMisc {
   uint64_t full[8];
   uint64_t empty[8];
   int32_t stage_ok[8];   // 1 = the stage holds valid K/V, 0 = its page was out of range
-  float wm[kDecWarps][16];
-  float wl[kDecWarps][16];
   int abort_flag;
 };
 
@@ -160,7 +158,6 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   DecMisc* misc = reinterpret_cast<DecMisc*>(smem + C::OFF_MISC);
-  float* oacc = reinterpret_cast<float*>(smem + C::OFF_OACC);
   volatile int* abort_flag = &misc->abort_flag;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -175,7 +172,6 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
     misc->abort_flag = 0;
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < 16 * D; i += blockDim.x) oacc[i] = 0.f;
   __syncthreads();
 
   if (warp == kDecWarps) {
@@ -265,14 +261,20 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       }
     }
   } else {
-    // ================= consumers
+    // ================= consumers.  Piece gp of the CTA's stream goes to warp gp % 4 and
+    // ring stage gp % NST, so each warp owns the stages w, w + 4, ...: every wait on a
+    // stage follows the same warp's wait on that stage's previous use, which keeps the
+    // phase parity unambiguous without any barrier between the warps.  Each warp keeps
+    // its own online-softmax state for the item and writes it as one partial (O
+    // normalised by its own sum, plus its log2-sum-exp); the merge kernel combines the
+    // partials, so the warps never wait for one another.
     const int g = lane >> 2;  // row (query head within the group) of the MMA fragments
     const int t = lane & 3;
     constexpr int NT = D / 8;  // n-tiles of the P V product
     const uint32_t ring = smem_u32(smem + C::OFF_RING);
     int gp_base = 0;
     bool ok = true;
-    for (int f = blockIdx.x; f < n_items; f += gridDim.x) {
+    for (int f = blockIdx.x; f < n_items && ok; f += gridDim.x) {
       const DecItem it = decode_item(a, f, item_info(a, f));
       const int npieces = (it.ntok + kDecTok - 1) / kDecTok;
       const int hq0 = it.kvh * a.group + it.hg * 16;
@@ -296,7 +298,8 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       for (int n = 0; n < NT; ++n) oc[n][0] = oc[n][1] = oc[n][2] = oc[n][3] = 0.f;
       float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows g and g+8
 
-      for (int i = warp; i < npieces && ok; i += kDecWarps) {
+      // this warp's pieces of the item: global piece indices gp with gp % 4 == warp
+      for (int i = (warp - gp_base % kDecWarps + kDecWarps) % kDecWarps; i < npieces; i += kDecWarps) {
         const int gp = gp_base + i;
         const int st = gp % C::NST;
         if (!mbar_wait(&misc->full[st], (gp / C::NST) & 1, abort_flag, a.timeout_ns)) {
@@ -383,58 +386,29 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
         if (lane == 0) mbar_arrive(&misc->empty[st]);
       }
       gp_base += npieces;
+      if (!ok) break;
 
-      // ---- merge the four warps' states for this item
+      // ---- this warp's partial for the item: O / l (rows < nrows) and log2-sum-exp
       l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
       l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-      if (t == 0) {
-        misc->wm[warp][g] = m0;
-        misc->wm[warp][g + 8] = m1;
-        misc->wl[warp][g] = l0;
-        misc->wl[warp][g + 8] = l1;
-      }
-      named_bar_sync(1, kDecWarps * 32);
-      float M0 = -INFINITY, M1 = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) {
-        M0 = fmaxf(M0, misc->wm[w][g]);
-        M1 = fmaxf(M1, misc->wm[w][g + 8]);
-      }
-      float L0 = 0.f, L1 = 0.f;
-#pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) {
-        if (misc->wm[w][g] != -INFINITY) L0 += misc->wl[w][g] * ex2(misc->wm[w][g] - M0);
-        if (misc->wm[w][g + 8] != -INFINITY) L1 += misc->wl[w][g + 8] * ex2(misc->wm[w][g + 8] - M1);
-      }
-      const float f0 = (m0 == -INFINITY || L0 == 0.f) ? 0.f : ex2(m0 - M0) / L0;
-      const float f1 = (m1 == -INFINITY || L1 == 0.f) ? 0.f : ex2(m1 - M1) / L1;
+      const float i0 = l0 > 0.f ? 1.f / l0 : 0.f;
+      const float i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+      const size_t pbase = (((size_t)it.s * a.max_chunks + it.c) * kDecWarps + warp) * a.Hq + hq0;
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
         const int col = n * 8 + 2 * t;
-        atomicAdd(&oacc[g * D + col], oc[n][0] * f0);
-        atomicAdd(&oacc[g * D + col + 1], oc[n][1] * f0);
-        atomicAdd(&oacc[(g + 8) * D + col], oc[n][2] * f1);
-        atomicAdd(&oacc[(g + 8) * D + col + 1], oc[n][3] * f1);
+        if (g < nrows)
+          *reinterpret_cast<float2*>(a.part_o + (pbase + g) * D + col) = make_float2(oc[n][0] * i0, oc[n][1] * i0);
+        if (g + 8 < nrows)
+          *reinterpret_cast<float2*>(a.part_o + (pbase + g + 8) * D + col) =
+              make_float2(oc[n][2] * i1, oc[n][3] * i1);
       }
-      named_bar_sync(1, kDecWarps * 32);
-      // write the partial: rows < nrows, normalised O and log2-sum-exp
-      const size_t pbase = ((size_t)it.s * a.max_chunks + it.c) * a.Hq + hq0;
-      for (int i = threadIdx.x; i < nrows * D; i += kDecWarps * 32) {
-        a.part_o[pbase * D + i] = oacc[i];
-        oacc[i] = 0.f;
+      if (t == 0) {
+        if (g < nrows) a.part_lse[pbase + g] = (l0 > 0.f) ? m0 + log2f(l0) : -INFINITY;
+        if (g + 8 < nrows) a.part_lse[pbase + g + 8] = (l1 > 0.f) ? m1 + log2f(l1) : -INFINITY;
       }
-      for (int i = nrows * D + threadIdx.x; i < 16 * D; i += kDecWarps * 32) oacc[i] = 0.f;
-      if (threadIdx.x < nrows) {
-        float M = -INFINITY, L = 0.f;
-        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, misc->wm[w][threadIdx.x]);
-        for (int w = 0; w < kDecWarps; ++w)
-          if (misc->wm[w][threadIdx.x] != -INFINITY) L += misc->wl[w][threadIdx.x] * ex2(misc->wm[w][threadIdx.x] - M);
-        a.part_lse[pbase + threadIdx.x] = (L > 0.f) ? M + log2f(L) : -INFINITY;
-      }
-      // leave together: every consumer warp takes the same decision here
-      if (named_bar_sync_or(1, kDecWarps * 32, !ok || *abort_flag)) break;
     }
   }
   __syncthreads();
@@ -455,12 +429,14 @@ __global__ void __launch_bounds__(256) attn_decode_merge_kernel(const __grid_con
   float acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  const int np = nch * kDecWarps;  // partials: one per (chunk, consumer warp)
+  const size_t p0 = (size_t)s * a.max_chunks * kDecWarps;
   float M = -INFINITY;
-  for (int c = 0; c < nch; ++c) M = fmaxf(M, a.part_lse[((size_t)s * a.max_chunks + c) * a.Hq + h]);
+  for (int c = 0; c < np; ++c) M = fmaxf(M, a.part_lse[(p0 + c) * a.Hq + h]);
   float L = 0.f;
   if (M != -INFINITY) {
-    for (int c = 0; c < nch; ++c) {
-      const size_t pi = ((size_t)s * a.max_chunks + c) * a.Hq + h;
+    for (int c = 0; c < np; ++c) {
+      const size_t pi = (p0 + c) * a.Hq + h;
       const float lc = a.part_lse[pi];
       if (lc == -INFINITY) continue;
       const float w = ex2(lc - M);

@@ -110,9 +110,10 @@ def test_decode_empty_batch_is_a_noop(lib):
 
 def test_workspace_size(lib):
     f = lib.attn_decode_paged_workspace_size
-    # 64 sequences, 64 query heads, d = 128, up to 2048 pages of 16 tokens: 16 chunks of 2048 tokens
+    # 64 sequences, 64 query heads, d = 128, up to 2048 pages of 16 tokens: 16 chunks of 2048
+    # tokens, one partial per (chunk, consumer warp) of each query head
     n = f(64, 64, 8, 128, 2048, 16)
-    parts = 64 * 16 * 64
+    parts = 64 * 16 * 4 * 64
     item_map = 64 * 16 * 16  # one 16-byte record per chunk
     assert n >= parts * 128 * 4 + parts * 4 + 65 * 4 + item_map
     assert n < parts * 129 * 4 + item_map + 4096
