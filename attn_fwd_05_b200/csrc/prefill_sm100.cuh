@@ -22,11 +22,14 @@
 //     idea for Blackwell).  TMEM: S0 | S1 | O0 | O1 = 128 + 128 + d + d columns.
 //   * Kernel "single" (d = 256): one Q tile, S double-buffered in TMEM (64 + 64 columns)
 //     next to O (256 columns), so the next S = Q K^T runs while the softmax works.
-//   * The reference of each row is its exact running maximum: whenever a block raises
-//     it, the row's O accumulator is rescaled in TMEM before the next P V.  The row's
-//     largest probability is then exactly 1 and its bf16 rounding is exact, which keeps
-//     sharply peaked rows accurate; O and the log-sum-exp are normalised by the one
+//   * d <= 128: the reference of each row is its exact running maximum: whenever a block
+//     raises it, the row's O accumulator is rescaled in TMEM before the next P V.  The
+//     row's largest probability is then exactly 1 and its bf16 rounding is exact, which
+//     keeps sharply peaked rows accurate; O and the log-sum-exp are normalised by the one
 //     fp32 sum of the probabilities.
+//   * d = 256: a rescale moves 256 TMEM columns, so the reference moves only when the
+//     maximum grows by more than 2^8, and O is normalised by the sum of the bf16-rounded
+//     probabilities (see softmax_row64_step).
 #pragma once
 
 #include "sm100_common.cuh"
@@ -144,11 +147,11 @@ __device__ __forceinline__ void rescale_o(uint32_t o_taddr, float alpha) {
   }
 }
 
-// Epilogue for one row: O / l to global (bf16 or fp32) and the log-sum-exp.
+// Epilogue for one row: O / lr to global (bf16 or fp32) and the log-sum-exp from l.
 template <int D>
 __device__ __forceinline__ void store_row(const FwdArgs& a, uint32_t o_taddr, bool have_o, bool valid, int b,
-                                          int hq, int q, float m, float l) {
-  const float inv = l > 0.f ? 1.0f / l : 0.f;
+                                          int hq, int q, float m, float l, float lr) {
+  const float inv = lr > 0.f ? 1.0f / lr : 0.f;
   const size_t row = ((size_t)b * a.Hq + hq) * (size_t)a.Nq + (size_t)(valid ? q : 0);
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {
@@ -253,12 +256,13 @@ __device__ __forceinline__ void issue_pv_split(uint32_t o_tmem, uint32_t s_tmem,
   }
 }
 
-// Three pairs of probabilities in every eight (kEmuMask) are computed on the FMA pipe
-// (exp2_fma2) instead of the exp unit: per block the exp unit alone would otherwise need
-// as many cycles as the tensor core, the bottleneck the FA4 page names for Blackwell
-// (section "Softmax distribué et émulé").  The split balances the exp unit against the
-// issue slots the polynomial costs.
-constexpr uint32_t kEmuMask = 0x00u;  // measured: FMA-pipe exps starve the MMA-issuing warp (see below)
+// A quarter of the probability pairs (kEmuMask) is computed on the FMA pipe (exp2_fma2)
+// instead of the exp unit: per block the exp unit alone needs as many cycles as the
+// tensor core, the bottleneck the FA4 page names for Blackwell (section "Softmax
+// distribué et émulé").  More than a quarter costs more issue slots than it saves: the
+// thread that issues the MMAs shares its scheduler with the softmax warps and is
+// starved by FMA-heavy neighbours.
+constexpr uint32_t kEmuMask = 0x88u;  // pairs 3 and 7 of each group of 8 (measured best of 0, 1/8, 2/8)
 
 // p = 2^(s * sl2 + nmu) for 32 pairs; the packed bf16 values go to TMEM at p_taddr in
 // two 16-column stores (so fewer of them are held in registers), (a0 + a1) gets the
@@ -653,9 +657,16 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
 // ====================================================================================
 
 // Softmax over the calling thread's whole 64-column row of one score block (one
-// warpgroup per tile).  Returns the factor for the row's O.
+// warpgroup per tile; d = 256).  With d = 256 an O rescale moves 256 TMEM columns, so
+// the row reference is kept until the maximum grows by more than 2^8 (p <= 256 then).
+// The largest probability is then not exactly 1, so two sums are kept: lr, the sum of
+// the bf16-rounded P that multiply V, normalises O (the rounding of a dominant
+// probability cancels in the ratio); l, the fp32 sum, gives the log-sum-exp.
+// Returns the factor for the row's O.
+constexpr float kStaleMaxSlack = 8.0f;  // log2 units
+
 __device__ __forceinline__ float softmax_row64_step(uint32_t s_taddr, bool masked, int col_limit, float sl2,
-                                                    float& m, float& l) {
+                                                    float& m, float& l, float& lr) {
   uint32_t r[64];
   tmem_ld32(s_taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
   tmem_ld32(s_taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
@@ -676,18 +687,30 @@ __device__ __forceinline__ float softmax_row64_step(uint32_t s_taddr, bool maske
   }
   const float mx = max3(x0, x1, fmaxf(s[62], s[63])) * sl2;
   float alpha = 1.0f;
-  if (mx > m) {
-    alpha = ex2(m - mx);
+  if (mx > m + kStaleMaxSlack) {  // false while nothing is visible (mx = -inf)
+    alpha = ex2(m - mx);          // 0 when m = -inf
     m = mx;
   }
   const float nmu = (m == -INFINITY) ? 0.0f : -m;
-  float a0 = 0.f, a1 = 0.f;
-  if (masked) {
-    exp_pairs<0u>(s, sl2, nmu, s_taddr, a0, a1);
-  } else {
-    exp_pairs<kEmuMask>(s, sl2, nmu, s_taddr, a0, a1);
+  float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint32_t P[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int i = 16 * half + k;
+      float y0, y1;
+      fma2(y0, y1, s[2 * i], s[2 * i + 1], sl2, sl2, nmu, nmu);
+      const float p0 = ex2(y0), p1 = ex2(y1);
+      add2(a0, a1, p0, p1);
+      const uint32_t w = pack_bf16x2(p0, p1);
+      P[k] = w;
+      add2(b0, b1, bf16lo_to_f32(w), bf16hi_to_f32(w));
+    }
+    tmem_st16(s_taddr + 16 * half, P);
   }
   l = l * alpha + (a0 + a1);
+  lr = lr * alpha + (b0 + b1);
   return alpha;
 }
 
@@ -698,7 +721,9 @@ struct SingleCfg {
   static constexpr int THREADS = 256;  // warp 0 TMA, warp 1 MMA, warps 4-7 softmax
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int NSTAGE = 4;
+  // 5 stages: S(j+2) needs K(j+2) right after P V(j), and with 4 stages that tile can
+  // only start loading once P V(j-1) has released its stage (225.5 KB of shared memory)
+  static constexpr int NSTAGE = 5;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NSTAGE * KV_BYTES;
@@ -852,7 +877,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
     const uint32_t o_addr = tmem + lane_off + C::COL_O;
     const int q = job.q0 + r;
     const int klim = row_key_limit(a, q);
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f, lr = 0.f;
     bool ok = true;
     for (int j = 0; j < nblk; ++j) {
       if (!mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag, a.timeout_ns)) {
@@ -862,7 +887,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
       tc_fence_after();
       const uint32_t s_addr = tmem + lane_off + ((j & 1) ? C::COL_S1 : C::COL_S0);
       const bool masked = block_needs_mask<BN>(a, job, j);
-      const float alpha = softmax_row64_step(s_addr, masked, klim - j * BN, a.scale_log2, m, l);
+      const float alpha = softmax_row64_step(s_addr, masked, klim - j * BN, a.scale_log2, m, l, lr);
       if (__any_sync(0xffffffffu, alpha != 1.0f) && j > 0) {
         // P V(j-2) finished before S(j) (issued after it), so o_done is in phase j-1 or
         // later and its parity names P V(j-1) without ambiguity
@@ -885,7 +910,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
       ok = mbar_wait(&bars->o_final, 0, abort_flag, a.timeout_ns);
       tc_fence_after();
     }
-    if (ok) store_row<D>(a, o_addr, have_o, r < job.rows, b, hq, q, m, l);
+    if (ok) store_row<D>(a, o_addr, have_o, r < job.rows, b, hq, q, m, l, lr);
   }
 
   tc_fence_before();
