@@ -38,6 +38,15 @@ Readings where the pages are silent (each one is listed in the design notes):
   aligned to the bottom-right corner; the pages only say a triangular mask is
   supported.  With Nq == Nk this is the usual j <= i.
 * a query row with no visible key returns O = 0 and LSE = -inf.
+* sliding window of w tokens (ranksignal.fr, "Trois idées reçues à écarter": attend
+  only to the last w tokens; polydesk.ai glossary, "FlashAttention et attention
+  block-sparse": a sliding window is one of the block patterns): key j is visible to
+  query i iff i' - w < j <= i' with i' = i + (Nk - Nq), the same bottom-right alignment
+  as the causal mask.
+* block-sparse mask (same glossary section: a mask over blocks of tokens says which
+  blocks attend to each other): blocks of 128 queries by 128 keys; block_mask[bq][bk]
+  nonzero means the queries of block bq see the keys of block bk; one mask for every
+  batch and head; optionally intersected with the causal mask.
 * LSE is the natural log of sum_j exp(scale * q.k_j) over visible keys.
 * GQA: query head h uses K/V head h // (Hq / Hkv) (contiguous groups).
 * paging: row s of the block table lists the pool pages of sequence s in
@@ -81,9 +90,33 @@ def causal_visible(rows: np.ndarray, nq: int, nk: int) -> np.ndarray:
     return j <= i + (nk - nq)
 
 
+MASK_BLOCK = 128  # block size of the block-sparse reading
+
+
+def visible_mask(rows: np.ndarray, nq: int, nk: int, causal: bool, window: int | None = None,
+                 block_mask=None) -> np.ndarray | None:
+    """Boolean [len(rows), nk] of visible keys, or None when every key is visible.
+
+    causal: j <= i + (nk - nq).  window: additionally j > i + (nk - nq) - window.
+    block_mask: [ceil(nq/128), ceil(nk/128)], nonzero = the block pair attends.
+    """
+    rows = np.asarray(rows)
+    vis = None
+    if causal or window is not None:
+        vis = causal_visible(rows, nq, nk)
+    if window is not None:
+        j = np.arange(nk)[None, :]
+        vis = vis & (j > rows[:, None] + (nk - nq) - window)
+    if block_mask is not None:
+        bm = np.asarray(block_mask) != 0
+        blk = bm[(rows // MASK_BLOCK)[:, None], (np.arange(nk) // MASK_BLOCK)[None, :]]
+        vis = blk if vis is None else (vis & blk)
+    return vis
+
+
 def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float, causal: bool,
                    rows: np.ndarray | None = None, nq: int | None = None,
-                   want_p: bool = False):
+                   want_p: bool = False, window: int | None = None, block_mask=None):
     """One head: the three materialised steps of [85pct-VRAM] "L'attention classique en 3 étapes".
 
     q: [R, d] query rows (absolute row indices ``rows`` among ``nq`` queries),
@@ -98,8 +131,9 @@ def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float, ca
         nq = R
     # step 1: scores S = scale * Q K^T  ([FA-glossary] formula; [FA-PA] uses sqrt(d_k))
     S = scale * (q @ k.T)
-    if causal:
-        S = np.where(causal_visible(rows, nq, nk), S, -np.inf)
+    vis = visible_mask(rows, nq, nk, causal, window, block_mask)
+    if vis is not None:
+        S = np.where(vis, S, -np.inf)
     # step 2: P = softmax(S) along each row, with the row maximum taken out first
     rowmax = S.max(axis=1) if nk > 0 else np.full(R, -np.inf)
     alive = np.isfinite(rowmax)              # rows with at least one visible key
@@ -118,13 +152,14 @@ def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float, ca
 
 
 def _head_job(args):
-    q, k, v, scale, causal, row_block = args
+    q, k, v, scale, causal, row_block, window, block_mask = args
     nq = q.shape[0]
     O = np.empty((nq, v.shape[1]))
     L = np.empty(nq)
     for r0 in range(0, nq, row_block):
         rows = np.arange(r0, min(nq, r0 + row_block))
-        O[rows], L[rows] = attention_head(q[rows], k, v, scale, causal, rows=rows, nq=nq)
+        O[rows], L[rows] = attention_head(q[rows], k, v, scale, causal, rows=rows, nq=nq, window=window,
+                                          block_mask=block_mask)
     return O, L
 
 
@@ -134,18 +169,21 @@ def kv_head_of(hq: int, Hq: int, Hkv: int) -> int:
 
 
 def attention(q, k, v, scale: float, causal: bool, row_block: int = 512,
-              threads: int | None = None):
+              threads: int | None = None, window: int | None = None, block_mask=None):
     """Full attention. q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] (bf16 tensors or arrays).
 
     Returns O [B,Hq,Nq,d] and LSE [B,Hq,Nq] as float64 arrays.  Heads run on a
-    thread pool; each head is the plain routine above.
+    thread pool; each head is the plain routine above.  ``window`` and ``block_mask``
+    add the sliding-window and block-sparse masks described in the module notes.
     """
     q, k, v = as_f64(q), as_f64(k), as_f64(v)
     B, Hq, Nq, _ = q.shape
     Hkv = k.shape[1]
     assert Hq % Hkv == 0, "Hq must be a multiple of Hkv"
+    if block_mask is not None and hasattr(block_mask, "cpu"):
+        block_mask = block_mask.cpu().numpy()
     jobs = [(q[b, h], k[b, kv_head_of(h, Hq, Hkv)], v[b, kv_head_of(h, Hq, Hkv)],
-             scale, causal, row_block) for b in range(B) for h in range(Hq)]
+             scale, causal, row_block, window, block_mask) for b in range(B) for h in range(Hq)]
     threads = threads or os.cpu_count() or 1
     if threads > 1 and len(jobs) > 1:
         ctx = threadpool_limits(1) if threadpool_limits is not None else _nullctx()
@@ -158,7 +196,7 @@ def attention(q, k, v, scale: float, causal: bool, row_block: int = 512,
     return O, L
 
 
-def attention_rows(q, k, v, scale: float, causal: bool, b: int, hq: int, rows):
+def attention_rows(q, k, v, scale: float, causal: bool, b: int, hq: int, rows, window=None, block_mask=None):
     """Selected query rows of one (batch, head), computed one by one from the full K/V.
 
     Used to check sampled outputs of full-size runs.  Same arithmetic as
@@ -171,7 +209,7 @@ def attention_rows(q, k, v, scale: float, causal: bool, b: int, hq: int, rows):
     qr = as_f64(q[b, hq][rows])
     kk = as_f64(k[b, kv])
     vv = as_f64(v[b, kv])
-    return attention_head(qr, kk, vv, scale, causal, rows=rows, nq=Nq)
+    return attention_head(qr, kk, vv, scale, causal, rows=rows, nq=Nq, window=window, block_mask=block_mask)
 
 
 class _nullctx:

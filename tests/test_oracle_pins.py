@@ -317,3 +317,66 @@ def test_a_transposed_product_would_be_caught():
     P = np.exp(S - S.max(1, keepdims=True))
     P /= P.sum(1, keepdims=True)
     assert np.abs(P @ v - bo).max() > 1e-3
+
+
+# ---------------------------------------------------------------- sliding window and block-sparse masks
+
+def _explicit_mask(nq, nk, causal, window=None, block=None):
+    m = torch.zeros(nq, nk, dtype=torch.bool)
+    for i in range(nq):
+        for j in range(nk):
+            ok = True
+            if causal or window is not None:
+                ok = j <= i + (nk - nq)
+            if window is not None:
+                ok = ok and j > i + (nk - nq) - window
+            if block is not None:
+                ok = ok and bool(block[i // 128][j // 128])
+            m[i, j] = ok
+    return m
+
+
+@pytest.mark.parametrize("nq,nk,w", [(40, 40, 7), (30, 50, 12), (50, 30, 5), (20, 20, 1), (33, 33, 100)])
+def test_window_matches_sdpa_with_explicit_mask(nq, nk, w):
+    q, k, v = randn(1, 2, nq, 8), randn(1, 2, nk, 8), randn(1, 2, nk, 8)
+    mask = _explicit_mask(nq, nk, True, window=w)
+    O, L = attention(q, k, v, 0.4, True, window=w, threads=1)
+    rows_alive = mask.any(dim=1).numpy()
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *(torch.from_numpy(x) for x in (q, k, v)), attn_mask=mask, scale=0.4).numpy()
+    np.testing.assert_allclose(O[..., rows_alive, :], ref[..., rows_alive, :], atol=1e-12)
+    assert np.all(O[..., ~rows_alive, :] == 0) and np.all(np.isneginf(L[..., ~rows_alive]))
+
+
+def test_window_of_one_returns_own_value_and_wide_window_is_causal():
+    q, k, v = randn(1, 1, 20, 6), randn(1, 1, 20, 6), randn(1, 1, 20, 6)
+    O, L = attention(q, k, v, 0.5, True, window=1, threads=1)
+    np.testing.assert_allclose(O[0, 0], v[0, 0], atol=1e-15)
+    np.testing.assert_allclose(L[0, 0], 0.5 * np.einsum("id,id->i", q[0, 0], k[0, 0]), atol=1e-13)
+    Ow, Lw = attention(q, k, v, 0.5, True, window=20, threads=1)
+    Oc, Lc = attention(q, k, v, 0.5, True, threads=1)
+    np.testing.assert_array_equal(Ow, Oc)
+    np.testing.assert_array_equal(Lw, Lc)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_mask_matches_sdpa_with_explicit_mask(causal):
+    nq, nk = 300, 400
+    bm = (np.random.default_rng(5).random(((nq + 127) // 128, (nk + 127) // 128)) > 0.4).astype(np.uint8)
+    bm[0, 0] = 1
+    q, k, v = randn(1, 2, nq, 8), randn(1, 2, nk, 8), randn(1, 2, nk, 8)
+    mask = _explicit_mask(nq, nk, causal, block=bm)
+    O, L = attention(q, k, v, 0.3, causal, block_mask=bm, threads=1)
+    alive = mask.any(dim=1).numpy()
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *(torch.from_numpy(x) for x in (q, k, v)), attn_mask=mask, scale=0.3).numpy()
+    np.testing.assert_allclose(O[..., alive, :], ref[..., alive, :], atol=1e-12)
+    assert np.all(O[..., ~alive, :] == 0) and np.all(np.isneginf(L[..., ~alive]))
+
+
+def test_full_block_mask_is_no_mask():
+    q, k, v = randn(1, 1, 200, 4), randn(1, 1, 300, 4), randn(1, 1, 300, 4)
+    O1, L1 = attention(q, k, v, 0.3, False, block_mask=np.ones((2, 3), np.uint8), threads=1)
+    O2, L2 = attention(q, k, v, 0.3, False, threads=1)
+    np.testing.assert_array_equal(O1, O2)
+    np.testing.assert_array_equal(L1, L2)
