@@ -31,6 +31,7 @@ SIGNATURES = {
     "attn_abi_version": (_I, []),
     "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P]),
     "attn_fwd_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P]),
+    "attn_fwd_masked": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _I, _P, _P]),
     "attn_decode_paged_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
     "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P,
                                ctypes.c_size_t, _P]),
@@ -98,10 +99,7 @@ def _dev(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int | None = None
     return t.data_ptr()
 
 
-def attn_fwd_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor | None,
-                causal: bool, scale: float, stream=None) -> None:
-    """Prefill forward; o is bf16 or fp32 [B, Hq, Nq, d], lse fp32 [B, Hq, Nq] or None."""
-    lib = load_library()
+def _fwd_shapes(q, k, v, o, lse):
     B, Hq, Nq, d = q.shape
     Hkv, Nk = k.shape[1], k.shape[2]
     if tuple(k.shape) != (B, Hkv, Nk, d) or tuple(v.shape) != tuple(k.shape):
@@ -116,11 +114,37 @@ def attn_fwd_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tens
         odt = DTYPE_F32
     else:
         raise TypeError("o must be bf16 or fp32")
-    st = lib.attn_fwd_ex(_dev(q, "q", torch.bfloat16, 4), _dev(k, "k", torch.bfloat16, 4),
-                         _dev(v, "v", torch.bfloat16, 4), _dev(o, "o", o.dtype, 4), odt,
-                         None if lse is None else _dev(lse, "lse", torch.float32, 3),
-                         B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), _stream(stream))
+    ptrs = (_dev(q, "q", torch.bfloat16, 4), _dev(k, "k", torch.bfloat16, 4), _dev(v, "v", torch.bfloat16, 4),
+            _dev(o, "o", o.dtype, 4), odt, None if lse is None else _dev(lse, "lse", torch.float32, 3))
+    return ptrs, (B, Hq, Hkv, Nq, Nk, d)
+
+
+def attn_fwd_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor | None,
+                causal: bool, scale: float, stream=None) -> None:
+    """Prefill forward; o is bf16 or fp32 [B, Hq, Nq, d], lse fp32 [B, Hq, Nq] or None."""
+    lib = load_library()
+    ptrs, dims = _fwd_shapes(q, k, v, o, lse)
+    st = lib.attn_fwd_ex(*ptrs, *dims, float(scale), int(bool(causal)), _stream(stream))
     _check(st, "attn_fwd_ex")
+
+
+def attn_fwd_masked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor | None,
+                    causal: bool, scale: float, window: int = 0, block_mask: torch.Tensor | None = None,
+                    stream=None) -> None:
+    """Prefill forward with a sliding window (window > 0, needs causal) and/or a
+    block-sparse map: uint8 [ceil(Nq/128), ceil(Nk/128)] on the device, nonzero =
+    the 128 x 128 block pair attends."""
+    lib = load_library()
+    ptrs, dims = _fwd_shapes(q, k, v, o, lse)
+    bm = None
+    if block_mask is not None:
+        Nq, Nk = dims[3], dims[4]
+        want = ((Nq + 127) // 128, (Nk + 127) // 128)
+        if tuple(block_mask.shape) != want:
+            raise ValueError(f"block_mask must be {want}")
+        bm = _dev(block_mask, "block_mask", torch.uint8, 2)
+    st = lib.attn_fwd_masked(*ptrs, *dims, float(scale), int(bool(causal)), int(window), bm, _stream(stream))
+    _check(st, "attn_fwd_masked")
 
 
 def attn_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:

@@ -208,10 +208,14 @@ const char* attn_status_string(int s) {
   }
 }
 
-attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, int o_dtype, float* lse, int B,
-                        int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, void* stream) {
+namespace {
+
+attn_status fwd_common(const void* q, const void* k, const void* v, void* o, int o_dtype, float* lse, int B, int Hq,
+                       int Hkv, int Nq, int Nk, int d, float scale, int causal, int window, const uint8_t* block_mask,
+                       void* stream) {
   if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (window < 0 || (window > 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
   if (o_dtype != ATTN_DTYPE_BF16 && o_dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.0f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
@@ -223,6 +227,13 @@ attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, in
       (lse != nullptr && !aligned(lse, 4)))
     return ATTN_ERR_ALIGNMENT;
   if ((long long)B * Hq > 0x7fffffffLL || (long long)B * Hkv > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  // block-sparse map: one byte per 128 x 128 block; a CTA keeps its visited blocks in a
+  // bounded shared-memory list (d <= 128) or bitmap (d = 256)
+  const long long nkt = ((long long)Nk + attn::kMaskBlock - 1) / attn::kMaskBlock;
+  if (block_mask != nullptr) {
+    const long long max_nkt = d <= 128 ? (long long)attn::kMaxVisits : 1024;
+    if (nkt > max_nkt) return ATTN_ERR_TOO_LARGE;
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int o_f32 = o_dtype == ATTN_DTYPE_F32;
 
@@ -252,11 +263,28 @@ attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, in
   a.pair_heads = (a.group % 2 == 0) ? 1 : 0;
   a.n_qtiles = (Nq + 127) / 128;
   a.timeout_ns = kDefaultTimeoutNs;
+  // a window wider than every row's visible prefix hides nothing
+  a.window = ((long long)window >= (long long)Nk + 1 || window == 0) ? 0 : window;
+  a.block_mask = block_mask;
+  a.nkt = (int)nkt;
   switch (d) {
     case 64: return launch_prefill<64>(a, st);
     case 128: return launch_prefill<128>(a, st);
     default: return launch_prefill<256>(a, st);
   }
+}
+
+}  // namespace
+
+attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, int o_dtype, float* lse, int B,
+                        int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, void* stream) {
+  return fwd_common(q, k, v, o, o_dtype, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, nullptr, stream);
+}
+
+attn_status attn_fwd_masked(const void* q, const void* k, const void* v, void* o, int o_dtype, float* lse, int B,
+                            int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, int window,
+                            const uint8_t* block_mask, void* stream) {
+  return fwd_common(q, k, v, o, o_dtype, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window, block_mask, stream);
 }
 
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,

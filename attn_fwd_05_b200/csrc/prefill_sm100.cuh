@@ -53,13 +53,22 @@ struct FwdArgs {
   int n_qtiles;      // ceil(Nq / 128)
   int n_units;
   uint64_t timeout_ns;
+  // masks beyond causal: window > 0 hides keys older than `window` tokens (with causal);
+  // block_mask (not null) is a [n_qtiles][nkt] map of 128x128 blocks, nonzero = visible
+  int window;
+  const uint8_t* block_mask;
+  int nkt;  // ceil(Nk / 128)
 };
+
+constexpr int kMaskBlock = 128;  // block size of the block-sparse map
+constexpr int kMaxVisits = 2048;  // blocks a CTA may visit under a block-sparse map
 
 struct TileJob {
   int hq;    // query head
   int q0;    // first query row of the tile
   int rows;  // valid rows (0 if the tile lies past Nq)
-  int nblk;  // KV blocks this tile visits
+  int jlo;   // first KV block the tile may visit
+  int jhi;   // one past the last KV block the tile may visit (jlo >= jhi: none)
 };
 
 template <int BN>
@@ -67,9 +76,10 @@ __device__ __forceinline__ TileJob make_tile(const FwdArgs& a, int hq, int q0) {
   TileJob t;
   t.hq = hq;
   t.q0 = q0;
+  t.jlo = 0;
+  t.jhi = 0;
   if (q0 >= a.Nq) {
     t.rows = 0;
-    t.nblk = 0;
     return t;
   }
   t.rows = min(128, a.Nq - q0);
@@ -81,16 +91,26 @@ __device__ __forceinline__ TileJob make_tile(const FwdArgs& a, int hq, int q0) {
     if (nkeys < 0) nkeys = 0;
     if (nkeys > a.Nk) nkeys = a.Nk;
   }
-  t.nblk = (int)((nkeys + BN - 1) / BN);
+  t.jhi = (int)((nkeys + BN - 1) / BN);
+  if (a.window > 0) {
+    // first visible key of the tile's first row: q0 + (Nk - Nq) - window + 1
+    long long first = (long long)q0 + a.Nk - a.Nq - a.window + 1;
+    if (first < 0) first = 0;
+    const long long jl = first / BN;
+    t.jlo = (int)(jl < t.jhi ? jl : t.jhi);
+  }
   return t;
 }
 
-// Does block j of this tile contain a masked key for some row of the tile?
+__device__ __forceinline__ int tile_nblk(const TileJob& t) { return t.rows > 0 ? max(0, t.jhi - t.jlo) : 0; }
+
+// Does block j of this tile contain a hidden key for some row of the tile?
 template <int BN>
 __device__ __forceinline__ bool block_needs_mask(const FwdArgs& a, const TileJob& t, int j) {
   long long hi = (long long)(j + 1) * BN;  // one past the block's last key
   if (hi > a.Nk) return true;
   if (a.causal && hi - 1 > (long long)t.q0 + a.Nk - a.Nq) return true;
+  if (a.window > 0 && (long long)j * BN < (long long)t.q0 + t.rows - 1 + a.Nk - a.Nq - a.window + 1) return true;
   return false;
 }
 
@@ -105,10 +125,109 @@ __device__ __forceinline__ int row_key_limit(const FwdArgs& a, int q) {
   return (int)lim;
 }
 
-// The MMA-issuing thread shares its scheduler with four busy softmax warps, so every
-// instruction it needs per MMA costs it dearly: descriptors are built once and each
-// k-step only adds its byte offset / 16 to the start-address field (offsets stay
-// inside one tile, so the 14-bit field never carries).
+// Smallest visible key index for query row q (0 without a window).
+__device__ __forceinline__ int row_key_low(const FwdArgs& a, int q) {
+  if (a.window <= 0) return 0;
+  long long lo = (long long)q + a.Nk - a.Nq - a.window + 1;
+  if (lo < 0) lo = 0;
+  if (lo > a.Nk) lo = a.Nk;
+  return (int)lo;
+}
+
+// The KV blocks a CTA visits: for causal / window / no masks, the union of its tiles'
+// ranges; under a block-sparse map, a list built in shared memory by one warp.
+struct VisitEntry {
+  uint16_t kb;   // KV block index
+  uint8_t part;  // bit t: tile t visits the block
+  uint8_t pad;
+};
+
+struct CtaPlan {
+  int nu;        // union steps
+  int ulo;       // first block of the union range (range plans)
+  int nv[2];     // visits of tile 0 and tile 1
+  int use_list;
+};
+
+template <int BN>
+__device__ __forceinline__ bool tile_visits(const FwdArgs& a, const TileJob& t, int kb) {
+  if (t.rows == 0 || kb < t.jlo || kb >= t.jhi) return false;
+  if (a.block_mask != nullptr)
+    return __ldg(&a.block_mask[(size_t)(t.q0 / kMaskBlock) * a.nkt + (kb * BN) / kMaskBlock]) != 0;
+  return true;
+}
+
+// Range plan, computed identically by every thread.
+__device__ __forceinline__ CtaPlan range_plan(const TileJob* tj, int ntiles) {
+  CtaPlan p;
+  int lo = 0x7fffffff, hi = 0;
+  for (int t = 0; t < 2; ++t) {
+    p.nv[t] = (t < ntiles) ? tile_nblk(tj[t]) : 0;
+    if (p.nv[t] > 0) {
+      lo = min(lo, tj[t].jlo);
+      hi = max(hi, tj[t].jhi);
+    }
+  }
+  p.ulo = (hi > 0) ? lo : 0;
+  p.nu = (hi > 0) ? hi - lo : 0;
+  p.use_list = 0;
+  return p;
+}
+
+// List plan for a block-sparse map: called by one whole warp; writes list[] and the
+// plan to shared memory.  Keeps at most kMaxVisits entries (the host bounds Nk).
+template <int BN>
+__device__ __forceinline__ void build_list_plan(const FwdArgs& a, const TileJob* tj, int ntiles, CtaPlan* plan,
+                                                VisitEntry* list) {
+  const int lane = threadIdx.x & 31;
+  const CtaPlan rp = range_plan(tj, ntiles);
+  int n = 0, n0 = 0, n1 = 0;
+  for (int base = 0; base < rp.nu; base += 32) {
+    const int kb = rp.ulo + base + lane;
+    const bool in = base + lane < rp.nu;
+    const bool v0 = in && tile_visits<BN>(a, tj[0], kb);
+    const bool v1 = in && ntiles > 1 && tile_visits<BN>(a, tj[1], kb);
+    const uint32_t m = __ballot_sync(0xffffffffu, v0 || v1);
+    const int rank = __popc(m & ((1u << lane) - 1u));
+    if ((v0 || v1) && n + rank < kMaxVisits) {
+      VisitEntry e;
+      e.kb = (uint16_t)kb;
+      e.part = (uint8_t)((v0 ? 1 : 0) | (v1 ? 2 : 0));
+      e.pad = 0;
+      list[n + rank] = e;
+    }
+    n += __popc(m);
+    n0 += __popc(__ballot_sync(0xffffffffu, v0));
+    n1 += __popc(__ballot_sync(0xffffffffu, v1));
+  }
+  if (lane == 0) {
+    plan->nu = min(n, kMaxVisits);
+    plan->ulo = 0;
+    plan->nv[0] = n0;
+    plan->nv[1] = n1;
+    plan->use_list = 1;
+  }
+}
+
+struct Visit {
+  int kb;
+  int part;
+};
+
+__device__ __forceinline__ Visit visit_at(const CtaPlan& p, const VisitEntry* list, const TileJob* tj, int u) {
+  Visit v;
+  if (p.use_list) {
+    const VisitEntry e = list[u];
+    v.kb = e.kb;
+    v.part = e.part;
+  } else {
+    v.kb = p.ulo + u;
+    v.part = ((p.nv[0] > 0 && v.kb >= tj[0].jlo && v.kb < tj[0].jhi) ? 1 : 0) |
+             ((p.nv[1] > 0 && v.kb >= tj[1].jlo && v.kb < tj[1].jhi) ? 2 : 0);
+  }
+  return v;
+}
+
 template <int D, int BN>
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t sQ, uint32_t sK) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, BN, 0, 0);
@@ -217,7 +336,9 @@ struct PingPongCfg {
   static constexpr int OFF_KV = 2 * Q_BYTES;
   static constexpr int OFF_RED = OFF_KV + NSTAGE * KV_BYTES;  // row-max / row-sum exchange
   static constexpr int RED_BYTES = 2 * 2 * 2 * 128 * 4 + 2 * 2 * 128 * 4;
-  static constexpr int OFF_BAR = OFF_RED + RED_BYTES;
+  static constexpr int OFF_PLAN = OFF_RED + RED_BYTES;  // CtaPlan + visit list (block-sparse maps)
+  static constexpr int PLAN_BYTES = 64 + kMaxVisits * 4;
+  static constexpr int OFF_BAR = OFF_PLAN + PLAN_BYTES;
   static constexpr int SMEM = OFF_BAR + 512 + 1024;  // barriers + 1 KB alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
@@ -295,7 +416,8 @@ __device__ __forceinline__ void exp_pairs(const float (&s)[64], float sl2, float
 //
 // The exchange barrier also ORs `stop` over both halves, so that they leave the block
 // loop at the same block (a half that left alone would hang the other on the barrier).
-__device__ __forceinline__ float softmax_half_step(uint32_t s_taddr, bool masked, int col_limit, float sl2,
+__device__ __forceinline__ float softmax_half_step(uint32_t s_taddr, bool masked, int col_limit, int col_low,
+                                                   float sl2,
                                                    float* xmax_mine, const float* xmax_other, int bar_id,
                                                    float& m, float& l, bool& stop) {
   uint32_t r[64];
@@ -308,7 +430,7 @@ __device__ __forceinline__ float softmax_half_step(uint32_t s_taddr, bool masked
   for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(r[c]);
   if (masked) {
 #pragma unroll
-    for (int c = 0; c < 64; ++c) s[c] = (c > col_limit) ? -INFINITY : s[c];
+    for (int c = 0; c < 64; ++c) s[c] = (c > col_limit || c < col_low) ? -INFINITY : s[c];
   }
   float x0 = max3(s[0], s[1], s[2]), x1 = max3(s[3], s[4], s[5]);
 #pragma unroll
@@ -402,13 +524,15 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   PingPongBars* bars = reinterpret_cast<PingPongBars*>(smem + C::OFF_BAR);
   PingPongRed* red = reinterpret_cast<PingPongRed*>(smem + C::OFF_RED);
+  CtaPlan* splan = reinterpret_cast<CtaPlan*>(smem + C::OFF_PLAN);
+  VisitEntry* vlist = reinterpret_cast<VisitEntry*>(smem + C::OFF_PLAN + 64);
   volatile int* abort_flag = &bars->abort_flag;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   // ---- work unit.  Causal: heaviest q-tiles first (longest-processing-time order).
-  // Non-causal: all units weigh the same; consecutive CTAs share a head so that the
+  // Otherwise: all units weigh about the same; consecutive CTAs share a head so that the
   // K/V tiles they all stream stay in L2.
   int b, kvh;
   TileJob tj[2];
@@ -445,7 +569,6 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
     }
     kvh = tj[0].hq / a.group;
   }
-  const int nblk = max(tj[0].nblk, tj[1].nblk);
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
@@ -467,21 +590,24 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
     tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
+  if (warp == 3 && a.block_mask != nullptr) build_list_plan<BN>(a, tj, 2, splan, vlist);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  const CtaPlan plan = (a.block_mask != nullptr) ? *splan : range_plan(tj, 2);
+  const int nu = plan.nu;
   const uint32_t tmem = bars->tmem_base;
   const uint32_t sQ[2] = {smem_u32(smem + C::OFF_Q), smem_u32(smem + C::OFF_Q + C::Q_BYTES)};
   const uint32_t sKV = smem_u32(smem + C::OFF_KV);
 
   if (warp == 0) {
-    // ================= TMA producer
+    // ================= TMA producer: Q tiles, then K and V of every visited block
     if (lane == 0) {
       tma_prefetch_map(&a.tm_q);
       tma_prefetch_map(&a.tm_k);
       tma_prefetch_map(&a.tm_v);
       for (int t = 0; t < 2; ++t) {
-        if (tj[t].nblk == 0) continue;
+        if (plan.nv[t] == 0) continue;
         mbar_arrive_expect_tx(&bars->q_full[t], C::Q_BYTES);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
@@ -491,7 +617,8 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
       const uint64_t pol = l2_policy_evict_last();
       int it = 0;
       bool ok = true;
-      for (int j = 0; j < nblk && ok; ++j) {
+      for (int u = 0; u < nu && ok; ++u) {
+        const int kb = visit_at(plan, vlist, tj, u).kb;
         for (int kv = 0; kv < 2 && ok; ++kv, ++it) {
           const int st = it % C::NSTAGE;
           const int use = it / C::NSTAGE;
@@ -504,79 +631,71 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
 #pragma unroll
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d_hint(smem + C::OFF_KV + st * C::KV_BYTES + c * (BN * 128), map, &bars->kv_full[st],
-                             c * 64, j * BN, b * a.Hkv + kvh, pol);
+                             c * 64, kb * BN, b * a.Hkv + kvh, pol);
         }
       }
       // drain: every copy issued must have landed before the CTA may exit
       for (int t = 0; t < 2; ++t)
-        if (tj[t].nblk > 0) mbar_wait(&bars->q_full[t], 0, abort_flag, a.timeout_ns, false);
+        if (plan.nv[t] > 0) mbar_wait(&bars->q_full[t], 0, abort_flag, a.timeout_ns, false);
       for (int st = 0; st < C::NSTAGE && st < it; ++st) {
         const int last_use = (it - 1 - st) / C::NSTAGE;  // index of the last fill of stage st
         mbar_wait(&bars->kv_full[st], last_use & 1, abort_flag, a.timeout_ns, false);
       }
     }
   } else if (warp == 1) {
-    // ================= MMA issuer.  Order per block j:
-    //   PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)
-    // so one tile's softmax overlaps the other tile's two MMAs.  S_t(j+1) overwrites
-    // the TMEM block that held P_t(j); it is issued after PV_t(j), and the tensor core
-    // executes one thread's MMAs in issue order.
-    if (lane == 0 && nblk > 0) {
+    // ================= MMA issuer.  Order per visited block u:
+    //   P V_0(u), S_0(u+1), P V_1(u), S_1(u+1)
+    // (each only for the tiles that visit the block) so one tile's softmax overlaps the
+    // other tile's two MMAs.  S_t(u+1) overwrites the TMEM block that held P_t(u); it is
+    // issued after P V_t(u), and the tensor core executes one thread's MMAs in issue
+    // order.  Barrier phases count each tile's own visits.
+    if (lane == 0 && nu > 0) {
       bool ok = true;
       for (int t = 0; t < 2 && ok; ++t)
-        if (tj[t].nblk > 0) ok = mbar_wait(&bars->q_full[t], 0, abort_flag, a.timeout_ns);
+        if (plan.nv[t] > 0) ok = mbar_wait(&bars->q_full[t], 0, abort_flag, a.timeout_ns);
       auto stage_of = [&](int it) { return it % C::NSTAGE; };
       auto parity_of = [&](int it) { return (uint32_t)((it / C::NSTAGE) & 1); };
+      int cnt[2] = {0, 0};  // visits of each tile issued so far (P V side)
+      Visit cur = visit_at(plan, vlist, tj, 0);
       if (ok) ok = mbar_wait(&bars->kv_full[stage_of(0)], parity_of(0), abort_flag, a.timeout_ns);
       if (ok) {
         tc_fence_after();
         for (int t = 0; t < 2; ++t) {
-          if (tj[t].nblk == 0) continue;
+          if (!(cur.part >> t & 1)) continue;
           issue_qk<D, BN>(tmem + (t ? C::COL_S1 : C::COL_S0), sQ[t], sKV + stage_of(0) * C::KV_BYTES);
           tc_commit(&bars->s_full[t]);
         }
         tc_commit(&bars->kv_empty[stage_of(0)]);
       }
-      for (int j = 0; j < nblk && ok; ++j) {
-        const int itV = 2 * j + 1, itK = 2 * j + 2;
+      for (int u = 0; u < nu && ok; ++u) {
+        const int itV = 2 * u + 1, itK = 2 * u + 2;
+        const bool more = u + 1 < nu;
+        const Visit nxt = more ? visit_at(plan, vlist, tj, u + 1) : Visit{0, 0};
         if (!mbar_wait(&bars->kv_full[stage_of(itV)], parity_of(itV), abort_flag, a.timeout_ns)) break;
+        if (more && !mbar_wait(&bars->kv_full[stage_of(itK)], parity_of(itK), abort_flag, a.timeout_ns)) break;
         const uint32_t sV = sKV + stage_of(itV) * C::KV_BYTES;
-        const bool next = (j + 1 < nblk);
-        bool k_ready = false;
         for (int t = 0; t < 2; ++t) {
           const uint32_t colS = t ? C::COL_S1 : C::COL_S0;
           const uint32_t colO = t ? C::COL_O1 : C::COL_O0;
-          if (j < tj[t].nblk) {
-            if (!mbar_wait(&bars->p_full[t], j & 1, abort_flag, a.timeout_ns)) {
+          if (cur.part >> t & 1) {
+            if (!mbar_wait(&bars->p_full[t], cnt[t] & 1, abort_flag, a.timeout_ns)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            issue_pv_split<D, BN>(tmem + colO, tmem + colS, sV, j > 0);
+            issue_pv_split<D, BN>(tmem + colO, tmem + colS, sV, cnt[t] > 0);
             tc_commit(&bars->o_done[t]);
-            if (j + 1 == tj[t].nblk) tc_commit(&bars->o_final[t]);
+            if (++cnt[t] == plan.nv[t]) tc_commit(&bars->o_final[t]);
           }
           if (t == 1) tc_commit(&bars->kv_empty[stage_of(itV)]);
-          if (next && j + 1 < tj[t].nblk) {
-            if (!k_ready) {
-              if (!mbar_wait(&bars->kv_full[stage_of(itK)], parity_of(itK), abort_flag, a.timeout_ns)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              k_ready = true;
-            }
+          if (more && (nxt.part >> t & 1)) {
             issue_qk<D, BN>(tmem + colS, sQ[t], sKV + stage_of(itK) * C::KV_BYTES);
             tc_commit(&bars->s_full[t]);
           }
         }
         if (!ok) break;
-        if (next) {
-          if (!k_ready) {  // no tile used K(j+1) (cannot happen when next is true, kept for safety)
-            if (!mbar_wait(&bars->kv_full[stage_of(itK)], parity_of(itK), abort_flag, a.timeout_ns)) break;
-          }
-          tc_commit(&bars->kv_empty[stage_of(itK)]);
-        }
+        if (more) tc_commit(&bars->kv_empty[stage_of(itK)]);
+        cur = nxt;
       }
       // every MMA must be finished before TMEM is released
       tc_commit(&bars->drain);
@@ -594,27 +713,37 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
     const uint32_t s_addr = tmem + lane_off + (t ? C::COL_S1 : C::COL_S0) + 64 * h;
     const uint32_t o_addr = tmem + lane_off + (t ? C::COL_O1 : C::COL_O0) + (D / 2) * h;
     const int q = job.q0 + r;
-    const int klim = row_key_limit(a, q) - 64 * h;  // limit relative to this half's first column
+    const int khi = row_key_limit(a, q) - 64 * h;  // limits relative to this half's first column
+    const int klo = row_key_low(a, q) - 64 * h;
     const int bar_id = 1 + t;
+    const int nv = plan.nv[t];
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     bool fail = false;  // a wait of this warp gave up; decided jointly at the next exchange
-    for (int j = 0; j < job.nblk; ++j) {
-      // both halves reach the exchange barrier of every block; an abort is decided
+    const bool use_list = plan.use_list != 0;
+    const int jlo = job.jlo;
+    int u = 0;  // list cursor
+    for (int k = 0; k < nv; ++k) {
+      int kb = jlo + k;  // range plan: the tile's blocks are contiguous
+      if (use_list) {
+        while (!(vlist[u].part >> t & 1)) ++u;
+        kb = vlist[u++].kb;
+      }
+      // both halves reach the exchange barrier of every visit; an abort is decided
       // jointly there
-      bool stop = fail || !mbar_wait(&bars->s_full[t], j & 1, abort_flag, a.timeout_ns) || *abort_flag;
+      bool stop = fail || !mbar_wait(&bars->s_full[t], k & 1, abort_flag, a.timeout_ns) || *abort_flag;
       tc_fence_after();
-      const bool masked = block_needs_mask<BN>(a, job, j);
-      const float alpha = softmax_half_step(s_addr, masked, klim - j * BN, a.scale_log2,
-                                            &red->xmax[t][j & 1][h][r], &red->xmax[t][j & 1][h ^ 1][r], bar_id,
+      const bool masked = block_needs_mask<BN>(a, job, kb);
+      const float alpha = softmax_half_step(s_addr, masked, khi - kb * BN, klo - kb * BN, a.scale_log2,
+                                            &red->xmax[t][k & 1][h][r], &red->xmax[t][k & 1][h ^ 1][r], bar_id,
                                             m, l, stop);
       if (stop) {
         fail = true;
         break;
       }
-      if (__any_sync(0xffffffffu, alpha != 1.0f) && j > 0) {
-        // O holds P V of blocks < j: wait for the last of those MMAs, then rescale
-        if (mbar_wait(&bars->o_done[t], (j - 1) & 1, abort_flag, a.timeout_ns)) {
+      if (__any_sync(0xffffffffu, alpha != 1.0f) && k > 0) {
+        // O holds P V of earlier visits: wait for the last of those MMAs, then rescale
+        if (mbar_wait(&bars->o_done[t], (k - 1) & 1, abort_flag, a.timeout_ns)) {
           tc_fence_after();
           rescale_cols<D / 2>(o_addr, alpha);
         } else {
@@ -627,7 +756,7 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
       if (lane == 0) mbar_arrive(&bars->p_full[t]);
     }
     ok = !fail;
-    const bool have_o = job.nblk > 0;
+    const bool have_o = nv > 0;
     if (ok && have_o) {
       ok = mbar_wait(&bars->o_final[t], 0, abort_flag, a.timeout_ns);
       tc_fence_after();
@@ -665,8 +794,8 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
 // Returns the factor for the row's O.
 constexpr float kStaleMaxSlack = 8.0f;  // log2 units
 
-__device__ __forceinline__ float softmax_row64_step(uint32_t s_taddr, bool masked, int col_limit, float sl2,
-                                                    float& m, float& l, float& lr) {
+__device__ __forceinline__ float softmax_row64_step(uint32_t s_taddr, bool masked, int col_limit, int col_low,
+                                                    float sl2, float& m, float& l, float& lr) {
   uint32_t r[64];
   tmem_ld32(s_taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
   tmem_ld32(s_taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
@@ -677,7 +806,7 @@ __device__ __forceinline__ float softmax_row64_step(uint32_t s_taddr, bool maske
   for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(r[c]);
   if (masked) {
 #pragma unroll
-    for (int c = 0; c < 64; ++c) s[c] = (c > col_limit) ? -INFINITY : s[c];
+    for (int c = 0; c < 64; ++c) s[c] = (c > col_limit || c < col_low) ? -INFINITY : s[c];
   }
   float x0 = max3(s[0], s[1], s[2]), x1 = max3(s[3], s[4], s[5]);
 #pragma unroll
@@ -743,7 +872,24 @@ struct SingleBars {
   uint64_t kv_empty[8];
   uint32_t tmem_base;
   int abort_flag;
+  uint32_t visible[32];  // block-sparse map row of the tile: bit mb = 128-key block mb
 };
+
+// Smallest block >= kb the tile visits (t.jhi if none).  bits: the tile's row of the
+// block-sparse map as a bitmap, or null when there is none.
+template <int BN>
+__device__ __forceinline__ int next_visit(const uint32_t* bits, const TileJob& t, int kb) {
+  if (kb < t.jlo) kb = t.jlo;
+  if (bits == nullptr) return kb < t.jhi ? kb : t.jhi;
+  while (kb < t.jhi) {
+    const int mb = kb * BN / kMaskBlock;
+    const uint32_t w = bits[mb >> 5] >> (mb & 31);
+    if (w & 1u) return kb;
+    const int skip = w ? __ffs(w) - 1 : 32 - (mb & 31);  // to the next set bit, or the next word
+    kb = (mb + skip) * (kMaskBlock / BN);
+  }
+  return t.jhi;
+}
 
 template <int D>
 __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_constant__ FwdArgs a) {
@@ -768,7 +914,6 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
     job = make_tile<BN>(a, hq, qt * 128);
   }
   const int kvh = hq / a.group;
-  const int nblk = job.nblk;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -790,15 +935,27 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
     tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
+  if (warp == 2 && a.block_mask != nullptr) {
+    // bitmap of the tile's map row (the host bounds nkt by 32 x 32)
+    const uint8_t* row = a.block_mask + (size_t)(job.q0 / kMaskBlock) * a.nkt;
+    for (int i = 0; i < 32; ++i) {
+      const int mb = 32 * i + lane;
+      const uint32_t w = __ballot_sync(0xffffffffu, mb < a.nkt && __ldg(&row[mb]) != 0);
+      if (lane == 0) bars->visible[i] = w;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const uint32_t sQ = smem_u32(smem + C::OFF_Q);
   const uint32_t sKV = smem_u32(smem + C::OFF_KV);
+  const uint32_t* bits = (a.block_mask != nullptr) ? bars->visible : nullptr;
+  const int kb0 = next_visit<BN>(bits, job, job.jlo);  // first visited block
+  const bool any = job.rows > 0 && kb0 < job.jhi;
 
   if (warp == 0) {
-    if (lane == 0 && nblk > 0) {
+    if (lane == 0 && any) {
       tma_prefetch_map(&a.tm_q);
       tma_prefetch_map(&a.tm_k);
       tma_prefetch_map(&a.tm_v);
@@ -809,7 +966,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
       const uint64_t pol = l2_policy_evict_last();
       int it = 0;
       bool ok = true;
-      for (int j = 0; j < nblk && ok; ++j) {
+      for (int kb = kb0; kb < job.jhi && ok; kb = next_visit<BN>(bits, job, kb + 1)) {
         for (int kv = 0; kv < 2; ++kv, ++it) {
           const int st = it % C::NSTAGE;
           const int use = it / C::NSTAGE;
@@ -822,7 +979,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
 #pragma unroll
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d_hint(smem + C::OFF_KV + st * C::KV_BYTES + c * (BN * 128), map, &bars->kv_full[st],
-                             c * 64, j * BN, b * a.Hkv + kvh, pol);
+                             c * 64, kb * BN, b * a.Hkv + kvh, pol);
         }
       }
       mbar_wait(&bars->q_full, 0, abort_flag, a.timeout_ns, false);
@@ -832,39 +989,44 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && nblk > 0) {
+    // Visit j: K at ring position 2j, V at 2j + 1; S(j) in TMEM block j & 1.  S(j + 2) is
+    // issued right after P V(j), which freed that block.
+    if (lane == 0 && any) {
       auto stage_of = [&](int it) { return it % C::NSTAGE; };
       auto parity_of = [&](int it) { return (uint32_t)((it / C::NSTAGE) & 1); };
       auto colS = [&](int j) { return (j & 1) ? C::COL_S1 : C::COL_S0; };
       bool ok = mbar_wait(&bars->q_full, 0, abort_flag, a.timeout_ns);
-      // S(0) and S(1) up front
-      for (int j = 0; j < 2 && j < nblk && ok; ++j) {
-        const int itK = 2 * j;
+      int nq = 0;      // Q K^T issued (visits 0 .. nq-1)
+      int kbq = kb0;   // block of the next Q K^T
+      for (; nq < 2 && kbq < job.jhi && ok; ++nq, kbq = next_visit<BN>(bits, job, kbq + 1)) {
+        const int itK = 2 * nq;
         if (!mbar_wait(&bars->kv_full[stage_of(itK)], parity_of(itK), abort_flag, a.timeout_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        issue_qk<D, BN>(tmem + colS(j), sQ, sKV + stage_of(itK) * C::KV_BYTES);
-        tc_commit(&bars->s_full[j & 1]);
+        issue_qk<D, BN>(tmem + colS(nq), sQ, sKV + stage_of(itK) * C::KV_BYTES);
+        tc_commit(&bars->s_full[nq & 1]);
         tc_commit(&bars->kv_empty[stage_of(itK)]);
       }
-      for (int j = 0; j < nblk && ok; ++j) {
+      for (int j = 0; j < nq && ok; ++j) {
         const int itV = 2 * j + 1;
         if (!mbar_wait(&bars->kv_full[stage_of(itV)], parity_of(itV), abort_flag, a.timeout_ns)) break;
         if (!mbar_wait(&bars->p_full[j & 1], (j >> 1) & 1, abort_flag, a.timeout_ns)) break;
         tc_fence_after();
         issue_pv<D, BN>(tmem + C::COL_O, tmem + colS(j), sKV + stage_of(itV) * C::KV_BYTES, j > 0);
         tc_commit(&bars->o_done);
-        if (j + 1 == nblk) tc_commit(&bars->o_final);
+        if (j + 1 == nq && kbq >= job.jhi) tc_commit(&bars->o_final);  // that was the last visit
         tc_commit(&bars->kv_empty[stage_of(itV)]);
-        if (j + 2 < nblk) {
-          const int itK = 2 * (j + 2);
+        if (kbq < job.jhi) {
+          const int itK = 2 * nq;  // nq == j + 2
           if (!mbar_wait(&bars->kv_full[stage_of(itK)], parity_of(itK), abort_flag, a.timeout_ns)) break;
           tc_fence_after();
-          issue_qk<D, BN>(tmem + colS(j), sQ, sKV + stage_of(itK) * C::KV_BYTES);
-          tc_commit(&bars->s_full[j & 1]);
+          issue_qk<D, BN>(tmem + colS(nq), sQ, sKV + stage_of(itK) * C::KV_BYTES);
+          tc_commit(&bars->s_full[nq & 1]);
           tc_commit(&bars->kv_empty[stage_of(itK)]);
+          ++nq;
+          kbq = next_visit<BN>(bits, job, kbq + 1);
         }
       }
       tc_commit(&bars->drain);
@@ -876,18 +1038,21 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t o_addr = tmem + lane_off + C::COL_O;
     const int q = job.q0 + r;
-    const int klim = row_key_limit(a, q);
+    const int khi = row_key_limit(a, q);
+    const int klo = row_key_low(a, q);
     float m = -INFINITY, l = 0.f, lr = 0.f;
     bool ok = true;
-    for (int j = 0; j < nblk; ++j) {
+    int j = 0;  // visits so far
+    for (int kb = any ? kb0 : job.jhi; kb < job.jhi; kb = next_visit<BN>(bits, job, kb + 1), ++j) {
       if (!mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag, a.timeout_ns)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const uint32_t s_addr = tmem + lane_off + ((j & 1) ? C::COL_S1 : C::COL_S0);
-      const bool masked = block_needs_mask<BN>(a, job, j);
-      const float alpha = softmax_row64_step(s_addr, masked, klim - j * BN, a.scale_log2, m, l, lr);
+      const bool masked = block_needs_mask<BN>(a, job, kb);
+      const float alpha =
+          softmax_row64_step(s_addr, masked, khi - kb * BN, klo - kb * BN, a.scale_log2, m, l, lr);
       if (__any_sync(0xffffffffu, alpha != 1.0f) && j > 0) {
         // P V(j-2) finished before S(j) (issued after it), so o_done is in phase j-1 or
         // later and its parity names P V(j-1) without ambiguity
@@ -903,9 +1068,9 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full[j & 1]);
     }
-    const bool have_o = nblk > 0;
+    const bool have_o = any;
     if (ok && have_o) {
-      // o_final, not o_done: the next Q K^T runs ahead of P V here, so P V(nblk-2) may
+      // o_final, not o_done: the next Q K^T runs ahead of P V here, so P V(j-2) may
       // still be in flight and o_done's parity could name an older completed phase
       ok = mbar_wait(&bars->o_final, 0, abort_flag, a.timeout_ns);
       tc_fence_after();

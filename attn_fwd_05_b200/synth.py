@@ -25,7 +25,7 @@ import torch
 _CHUNK = 1 << 24
 
 # stream ids: one independent generator per tensor
-_Q, _K, _V, _LENS, _PERM = 1, 2, 3, 4, 5
+_Q, _K, _V, _LENS, _PERM, _MASK = 1, 2, 3, 4, 5, 6
 
 
 @dataclass(frozen=True)
@@ -167,6 +167,14 @@ def decode_inputs(shape: DecodeShape, seed: int, seq_lens: np.ndarray | None = N
     return PagedKV(q=q, k_pool=k_pool, v_pool=v_pool,
                    block_table=torch.from_numpy(table),
                    seq_lens=torch.from_numpy(seq_lens.copy()), page_size=s.page_size)
+
+
+def block_mask(Nq: int, Nk: int, density: float, seed: int, block: int = 128) -> torch.Tensor:
+    """Seeded block-sparse map: uint8 [ceil(Nq/block), ceil(Nk/block)], each entry 1
+    with probability ``density`` (independently), else 0."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, _MASK, 0])))
+    shape = ((Nq + block - 1) // block, (Nk + block - 1) // block)
+    return torch.from_numpy((rng.random(shape) < density).astype(np.uint8))
 
 
 def default_scale(d: int) -> float:

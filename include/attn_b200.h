@@ -49,7 +49,8 @@ typedef enum attn_status {
   ATTN_ERR_BAD_PAGE = 6,        /* a block-table entry in use lies outside [0, num_pages) */
   ATTN_ERR_WORKSPACE = 7,       /* workspace null or smaller than attn_decode_paged_workspace_size */
   ATTN_ERR_TOO_LARGE = 8        /* attn_decode_paged_noalloc: the call needs more scratch than the
-                                   library's static scratch holds */
+                                   library's static scratch holds; attn_fwd_masked: Nk is past
+                                   the bound its block-sparse map allows */
 } attn_status;
 
 typedef enum attn_dtype {
@@ -100,6 +101,36 @@ attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, in
                         int causal, void* stream);
 
 /*
+ * attn_fwd_masked — attn_fwd_ex with two more masks, applied on top of the causal
+ * one.  A CTA skips the key blocks its rows cannot see, so both masks also save work.
+ *
+ * Sources: ranksignal.fr, "Trois idées reçues à écarter" (a sliding window: each token
+ * attends only to the most recent keys); polydesk.ai glossary "FlashAttention", section
+ * "FlashAttention et attention block-sparse" (a mask over blocks of tokens says which
+ * blocks attend to each other; sliding windows are one such pattern).
+ *
+ *   causal      0 or 1, as in attn_fwd.
+ *   window      0 = no window.  window >= 1 requires causal = 1: query i then sees key
+ *               j iff i' - window < j <= i' with i' = i + (Nk - Nq), i.e. the `window`
+ *               most recent keys up to its own position, same bottom-right alignment
+ *               as the causal mask.  window = 1 keeps the diagonal only.
+ *   block_mask  NULL = no block mask, else device, uint8 [ceil(Nq/128), ceil(Nk/128)]
+ *               row-major, read-only: entry [bq][bk] nonzero lets queries
+ *               128*bq .. 128*bq+127 see keys 128*bk .. 128*bk+127.  One map serves
+ *               every batch and head.  It is intersected with the causal mask and
+ *               the window.  Bound: ceil(Nk/128) <= 2048 for d <= 128 and <= 1024
+ *               for d = 256 (else ATTN_ERR_TOO_LARGE).
+ *
+ * A row with no visible key gets O = 0 and lse = -inf.  Other arguments, layouts and
+ * errors are those of attn_fwd_ex; window < 0, or window > 0 with causal = 0, gives
+ * ATTN_ERR_INVALID_ARG.
+ */
+attn_status attn_fwd_masked(const void* q, const void* k, const void* v, void* o, int o_dtype,
+                            float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                            float scale, int causal, int window, const uint8_t* block_mask,
+                            void* stream);
+
+/*
  * attn_decode_paged_workspace_size — bytes of scratch attn_decode_paged needs for
  * these sizes (fp32 partial outputs and partial log-sum-exps of the split-K pass).
  * Returns 0 for sizes attn_decode_paged would reject.
@@ -126,7 +157,8 @@ size_t attn_decode_paged_workspace_size(int num_seqs, int Hq, int Hkv, int d,
  *                [0, max_pages_per_seq*page_size]; the query attends to all of them.
  *   o            device, bf16 [num_seqs, Hq, d]   (written)
  *   lse          device, fp32 [num_seqs, Hq] or NULL (written when not NULL)
- *   page_size    16, 32 or 64;  d: 64, 128 or 256;  Hq % Hkv == 0 and Hq/Hkv <= 16.
+ *   page_size    16, 32 or 64;  d: 64, 128 or 256;  Hq % Hkv == 0 (query heads of
+ *                a KV head are handled 16 at a time).
  *   workspace    device scratch of at least attn_decode_paged_workspace_size(...) bytes,
  *                owned by the caller; its contents need no initialisation and are
  *                overwritten.  Two calls in flight at once need two workspaces.

@@ -87,6 +87,28 @@ def test_fwd_empty_work_is_a_noop(lib):
     assert fwd(lib, B=0, q=None, o=None) == OK
 
 
+def fwd_masked(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Hq=4, Hkv=2, Nq=16, Nk=16, d=128, scale=0.1,
+               causal=1, window=0, block_mask=None, odt=0):
+    return lib.attn_fwd_masked(q, k, v, o, odt, lse, B, Hq, Hkv, Nq, Nk, d, ctypes.c_float(scale), causal,
+                               window, block_mask, None)
+
+
+TOO_LARGE = 8
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(window=-1), INVALID), (dict(window=8, causal=0), INVALID), (dict(causal=3), INVALID),
+    (dict(block_mask=FAKE, Nk=2048 * 128 + 1), TOO_LARGE), (dict(block_mask=FAKE, d=256, Nk=1024 * 128 + 1), TOO_LARGE),
+    (dict(d=80), UNSUPPORTED), (dict(q=None), INVALID), (dict(k=FAKE + 4), ALIGN),
+])
+def test_fwd_masked_rejects_bad_arguments(lib, kw, code):
+    assert fwd_masked(lib, **kw) == code
+
+
+def test_fwd_masked_empty_work_is_a_noop(lib):
+    assert fwd_masked(lib, Nq=0, q=None, o=None, window=4) == OK
+
+
 def dec(lib, q=FAKE, kp=FAKE, vp=FAKE, bt=FAKE, sl=FAKE, ps=16, o=FAKE, lse=None, S=4, Hq=8, Hkv=2, d=128,
         npages=10, maxp=8, scale=0.1, ws=FAKE, wsb=1 << 30):
     return lib.attn_decode_paged(q, kp, vp, bt, sl, ps, o, lse, S, Hq, Hkv, d, npages, maxp,
