@@ -95,12 +95,14 @@ attn_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D>
+template <int D, bool MASKS>
 attn_status launch_prefill(attn::FwdArgs& a, cudaStream_t st) {
+  // shared-memory slots: 0-2 plain prefill, 3-5 decode, 6-8 masked prefill
+  const int slot = (D == 64 ? 0 : (D == 128 ? 1 : 2)) + (MASKS ? 6 : 0);
   if constexpr (D <= 128) {
     using C = attn::PingPongCfg<D>;
-    auto k = attn::attn_fwd_pingpong_kernel<D>;
-    if (!ensure_smem(k, C::SMEM, D == 64 ? 0 : 1)) return ATTN_ERR_CUDA;
+    auto k = attn::attn_fwd_pingpong_kernel<D, MASKS>;
+    if (!ensure_smem(k, C::SMEM, slot)) return ATTN_ERR_CUDA;
     const long long qp = (a.n_qtiles + 1) / 2;
     const long long units = a.pair_heads ? (long long)a.B * (a.Hq / 2) * a.n_qtiles : (long long)a.B * a.Hq * qp;
     if (units <= 0 || units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
@@ -108,8 +110,8 @@ attn_status launch_prefill(attn::FwdArgs& a, cudaStream_t st) {
     k<<<(unsigned)units, C::THREADS, C::SMEM, st>>>(a);
   } else {
     using C = attn::SingleCfg<D>;
-    auto k = attn::attn_fwd_single_kernel<D>;
-    if (!ensure_smem(k, C::SMEM, 2)) return ATTN_ERR_CUDA;
+    auto k = attn::attn_fwd_single_kernel<D, MASKS>;
+    if (!ensure_smem(k, C::SMEM, slot)) return ATTN_ERR_CUDA;
     const long long units = (long long)a.B * a.Hq * a.n_qtiles;
     if (units <= 0 || units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
     a.n_units = (int)units;
@@ -267,10 +269,11 @@ attn_status fwd_common(const void* q, const void* k, const void* v, void* o, int
   a.window = ((long long)window >= (long long)Nk + 1 || window == 0) ? 0 : window;
   a.block_mask = block_mask;
   a.nkt = (int)nkt;
+  const bool masks = a.window > 0 || a.block_mask != nullptr;
   switch (d) {
-    case 64: return launch_prefill<64>(a, st);
-    case 128: return launch_prefill<128>(a, st);
-    default: return launch_prefill<256>(a, st);
+    case 64: return masks ? launch_prefill<64, true>(a, st) : launch_prefill<64, false>(a, st);
+    case 128: return masks ? launch_prefill<128, true>(a, st) : launch_prefill<128, false>(a, st);
+    default: return masks ? launch_prefill<256, true>(a, st) : launch_prefill<256, false>(a, st);
   }
 }
 

@@ -71,7 +71,7 @@ struct TileJob {
   int jhi;   // one past the last KV block the tile may visit (jlo >= jhi: none)
 };
 
-template <int BN>
+template <int BN, bool MASKS>
 __device__ __forceinline__ TileJob make_tile(const FwdArgs& a, int hq, int q0) {
   TileJob t;
   t.hq = hq;
@@ -92,7 +92,7 @@ __device__ __forceinline__ TileJob make_tile(const FwdArgs& a, int hq, int q0) {
     if (nkeys > a.Nk) nkeys = a.Nk;
   }
   t.jhi = (int)((nkeys + BN - 1) / BN);
-  if (a.window > 0) {
+  if (MASKS && a.window > 0) {
     // first visible key of the tile's first row: q0 + (Nk - Nq) - window + 1
     long long first = (long long)q0 + a.Nk - a.Nq - a.window + 1;
     if (first < 0) first = 0;
@@ -102,15 +102,13 @@ __device__ __forceinline__ TileJob make_tile(const FwdArgs& a, int hq, int q0) {
   return t;
 }
 
-__device__ __forceinline__ int tile_nblk(const TileJob& t) { return t.rows > 0 ? max(0, t.jhi - t.jlo) : 0; }
-
 // Does block j of this tile contain a hidden key for some row of the tile?
-template <int BN>
+template <int BN, bool MASKS>
 __device__ __forceinline__ bool block_needs_mask(const FwdArgs& a, const TileJob& t, int j) {
   long long hi = (long long)(j + 1) * BN;  // one past the block's last key
   if (hi > a.Nk) return true;
   if (a.causal && hi - 1 > (long long)t.q0 + a.Nk - a.Nq) return true;
-  if (a.window > 0 && (long long)j * BN < (long long)t.q0 + t.rows - 1 + a.Nk - a.Nq - a.window + 1) return true;
+  if (MASKS && a.window > 0 && (long long)j * BN < (long long)t.q0 + t.rows - 1 + a.Nk - a.Nq - a.window + 1) return true;
   return false;
 }
 
@@ -134,98 +132,41 @@ __device__ __forceinline__ int row_key_low(const FwdArgs& a, int q) {
   return (int)lo;
 }
 
-// The KV blocks a CTA visits: for causal / window / no masks, the union of its tiles'
-// ranges; under a block-sparse map, a list built in shared memory by one warp.
-struct VisitEntry {
-  uint16_t kb;   // KV block index
-  uint8_t part;  // bit t: tile t visits the block
-  uint8_t pad;
-};
-
-struct CtaPlan {
-  int nu;        // union steps
-  int ulo;       // first block of the union range (range plans)
-  int nv[2];     // visits of tile 0 and tile 1
-  int use_list;
-};
-
+// Does the tile visit KV block kb?  bits: the tile's row of the block-sparse map as a
+// bitmap (bit mb = keys 128 mb .. 128 mb + 127), or null when there is none.
 template <int BN>
-__device__ __forceinline__ bool tile_visits(const FwdArgs& a, const TileJob& t, int kb) {
-  if (t.rows == 0 || kb < t.jlo || kb >= t.jhi) return false;
-  if (a.block_mask != nullptr)
-    return __ldg(&a.block_mask[(size_t)(t.q0 / kMaskBlock) * a.nkt + (kb * BN) / kMaskBlock]) != 0;
-  return true;
+__device__ __forceinline__ bool tile_visits(const uint32_t* bits, const TileJob& t, int kb) {
+  if (kb < t.jlo || kb >= t.jhi) return false;
+  if (bits == nullptr) return true;
+  const int mb = kb * BN / kMaskBlock;
+  return (bits[mb >> 5] >> (mb & 31)) & 1u;
 }
 
-// Range plan, computed identically by every thread.
-__device__ __forceinline__ CtaPlan range_plan(const TileJob* tj, int ntiles) {
-  CtaPlan p;
-  int lo = 0x7fffffff, hi = 0;
-  for (int t = 0; t < 2; ++t) {
-    p.nv[t] = (t < ntiles) ? tile_nblk(tj[t]) : 0;
-    if (p.nv[t] > 0) {
-      lo = min(lo, tj[t].jlo);
-      hi = max(hi, tj[t].jhi);
-    }
+// Smallest block >= kb the tile visits (t.jhi if none).
+template <int BN>
+__device__ __forceinline__ int next_visit(const uint32_t* bits, const TileJob& t, int kb) {
+  if (kb < t.jlo) kb = t.jlo;
+  if (bits == nullptr) return kb < t.jhi ? kb : t.jhi;
+  while (kb < t.jhi) {
+    const int mb = kb * BN / kMaskBlock;
+    const uint32_t w = bits[mb >> 5] >> (mb & 31);
+    if (w & 1u) return kb;
+    const int skip = w ? __ffs(w) - 1 : 32 - (mb & 31);  // to the next set bit, or the next word
+    kb = (mb + skip) * (kMaskBlock / BN);
   }
-  p.ulo = (hi > 0) ? lo : 0;
-  p.nu = (hi > 0) ? hi - lo : 0;
-  p.use_list = 0;
-  return p;
+  return t.jhi;
 }
 
-// List plan for a block-sparse map: called by one whole warp; writes list[] and the
-// plan to shared memory.  Keeps at most kMaxVisits entries (the host bounds Nk).
-template <int BN>
-__device__ __forceinline__ void build_list_plan(const FwdArgs& a, const TileJob* tj, int ntiles, CtaPlan* plan,
-                                                VisitEntry* list) {
+// One warp writes the tile's row of the block-sparse map as a bitmap of nwords words.
+__device__ __forceinline__ void build_row_bitmap(const FwdArgs& a, const TileJob& t, uint32_t* bits, int nwords) {
   const int lane = threadIdx.x & 31;
-  const CtaPlan rp = range_plan(tj, ntiles);
-  int n = 0, n0 = 0, n1 = 0;
-  for (int base = 0; base < rp.nu; base += 32) {
-    const int kb = rp.ulo + base + lane;
-    const bool in = base + lane < rp.nu;
-    const bool v0 = in && tile_visits<BN>(a, tj[0], kb);
-    const bool v1 = in && ntiles > 1 && tile_visits<BN>(a, tj[1], kb);
-    const uint32_t m = __ballot_sync(0xffffffffu, v0 || v1);
-    const int rank = __popc(m & ((1u << lane) - 1u));
-    if ((v0 || v1) && n + rank < kMaxVisits) {
-      VisitEntry e;
-      e.kb = (uint16_t)kb;
-      e.part = (uint8_t)((v0 ? 1 : 0) | (v1 ? 2 : 0));
-      e.pad = 0;
-      list[n + rank] = e;
-    }
-    n += __popc(m);
-    n0 += __popc(__ballot_sync(0xffffffffu, v0));
-    n1 += __popc(__ballot_sync(0xffffffffu, v1));
+  const uint8_t* row = a.block_mask + (size_t)(t.q0 / kMaskBlock) * a.nkt;
+  for (int i = 0; i < nwords; ++i) {
+    const int mb = 32 * i + lane;
+    const bool v = t.rows > 0 && mb < a.nkt && __ldg(&row[mb]) != 0;
+    const uint32_t w = __ballot_sync(0xffffffffu, v);
+    if (lane == 0) bits[i] = w;
   }
-  if (lane == 0) {
-    plan->nu = min(n, kMaxVisits);
-    plan->ulo = 0;
-    plan->nv[0] = n0;
-    plan->nv[1] = n1;
-    plan->use_list = 1;
-  }
-}
-
-struct Visit {
-  int kb;
-  int part;
-};
-
-__device__ __forceinline__ Visit visit_at(const CtaPlan& p, const VisitEntry* list, const TileJob* tj, int u) {
-  Visit v;
-  if (p.use_list) {
-    const VisitEntry e = list[u];
-    v.kb = e.kb;
-    v.part = e.part;
-  } else {
-    v.kb = p.ulo + u;
-    v.part = ((p.nv[0] > 0 && v.kb >= tj[0].jlo && v.kb < tj[0].jhi) ? 1 : 0) |
-             ((p.nv[1] > 0 && v.kb >= tj[1].jlo && v.kb < tj[1].jhi) ? 2 : 0);
-  }
-  return v;
 }
 
 template <int D, int BN>
@@ -313,16 +254,19 @@ __device__ __forceinline__ void store_row(const FwdArgs& a, uint32_t o_taddr, bo
 // ====================================================================================
 //
 // Warp roles (640 threads): warp 0 issues TMA loads, warp 1 issues the MMAs, warps 2-3
-// idle, warps 4-19 are four softmax warpgroups: tile t, column half h handled by
-// warpgroup 1 + 2t + h.  Each softmax thread owns one query row of its tile and 64 of
-// the 128 score columns of a block; the two halves of a row exchange their block
-// maxima through shared memory, so both apply the same reference.  Two warps per
-// scheduler work on a tile's softmax at once, which keeps the exp unit busy while the
-// other warp issues its arithmetic.
+// turn a block-sparse map into per-tile bitmaps (else idle), warps 4-19 are four
+// softmax warpgroups: tile t, column half h handled by warpgroup 1 + 2t + h.  Each
+// softmax thread owns one query row of its tile and 64 of the 128 score columns of a
+// block; the two halves of a row exchange their block maxima through shared memory,
+// so both apply the same reference.
 //
-// P is written over the half's own score columns (keys 64h..64h+63 of the block go
-// to TMEM columns 64h..64h+31 of the S block), so neither half can overwrite scores the
-// other still has to read.
+// P goes to shared memory (128-byte swizzled, K-major: the A operand of P V), not back
+// over S.  So S_t is free as soon as the softmax has read it into registers, and the
+// next S_t = Q_t K^T runs while the softmax still works on the current block: each
+// tile's softmax steps follow one another without waiting for the tensor core, and
+// the two tiles' softmaxes share the SM.  The MMA order per visited block u is
+// S_0(u+1), S_1(u+1), P V_0(u), P V_1(u); the K/V ring is filled in the same order
+// (K of block u+1 before V of block u).
 
 template <int D>
 struct PingPongCfg {
@@ -330,24 +274,28 @@ struct PingPongCfg {
   static constexpr int BN = 128;
   static constexpr int THREADS = 640;
   static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int P_BYTES = BM * BN * 2;
   static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int NSTAGE = (D == 64) ? 8 : 4;  // K and V tiles share the ring
+  static constexpr int NSTAGE = (D == 64) ? 8 : 3;  // K and V tiles share the ring
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = 2 * Q_BYTES;
-  static constexpr int OFF_RED = OFF_KV + NSTAGE * KV_BYTES;  // row-max / row-sum exchange
-  static constexpr int RED_BYTES = 2 * 2 * 2 * 128 * 4 + 2 * 2 * 128 * 4;
-  static constexpr int OFF_PLAN = OFF_RED + RED_BYTES;  // CtaPlan + visit list (block-sparse maps)
-  static constexpr int PLAN_BYTES = 64 + kMaxVisits * 4;
-  static constexpr int OFF_BAR = OFF_PLAN + PLAN_BYTES;
-  static constexpr int SMEM = OFF_BAR + 512 + 1024;  // barriers + 1 KB alignment slack
+  static constexpr int OFF_P = 2 * Q_BYTES;
+  static constexpr int OFF_KV = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_XMAX = OFF_KV + NSTAGE * KV_BYTES;  // block maxima [tile][half][row]
+  static constexpr int OFF_BAR = OFF_XMAX + 2 * 2 * 128 * 4;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int OFF_BITS = OFF_BAR + BAR_BYTES;  // block-sparse bitmaps [tile][64 words]
+  static constexpr int BITS_WORDS = kMaxVisits / 32;
+  static constexpr int SMEM = OFF_BITS + 2 * BITS_WORDS * 4;  // no alignment slack: the base is 1 KB aligned
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
+  static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
 struct PingPongBars {
   uint64_t q_full[2];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
+  uint64_t s_full[2];   // S_t of the tile's next visit is in TMEM
+  uint64_t s_free[2];   // the tile's softmax has read S_t and exchanged its maxima (8 warps)
+  uint64_t p_full[2];   // P_t is in shared memory and O_t is rescaled (8 warps)
   uint64_t o_done[2];   // one phase per P V of the tile
   uint64_t o_final[2];  // one phase: the tile's last P V is done
   uint64_t drain;
@@ -356,24 +304,20 @@ struct PingPongBars {
   uint32_t tmem_base;
   int abort_flag;
 };
+static_assert(sizeof(PingPongBars) <= PingPongCfg<128>::BAR_BYTES, "barrier area");
 
-// Exchange area: block maxima [tile][block parity][half][row] and final row sums
-// [tile][half][row].
-struct PingPongRed {
-  float xmax[2][2][2][128];
-  float sums[2][2][128];
-};
-
-// P V for one tile: k-step kk covers keys 16kk..16kk+15, whose packed P sits at TMEM
-// column 64*(kk/4) + 8*(kk%4) of the S block (each column half keeps its own P).
+// O_t += P_t V with P from shared memory: k-step kk covers keys 16kk..16kk+15 (64-key
+// chunk kk/4 of the K-major P tile, 32 bytes per step within it).
 template <int D, int BN>
-__device__ __forceinline__ void issue_pv_split(uint32_t o_tmem, uint32_t s_tmem, uint32_t sV, bool accumulate) {
+__device__ __forceinline__ void issue_pv_ss(uint32_t o_tmem, uint32_t sP, uint32_t sV, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+  const uint64_t da0 = smem_desc_sw128(sP, 16, 1024);
   const uint64_t db0 = smem_desc_sw128(sV, BN * 128, 1024);
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk) {
+    const uint64_t da = da0 + (uint64_t)((((kk >> 2) * (128 * 128)) + (kk & 3) * 32) >> 4);
     const uint64_t db = db0 + (uint64_t)((kk * (16 * 128)) >> 4);
-    mma_ts(o_tmem, s_tmem + (kk >> 2) * 64 + (kk & 3) * 8, db, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    mma_ss(o_tmem, da, db, idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -385,52 +329,52 @@ __device__ __forceinline__ void issue_pv_split(uint32_t o_tmem, uint32_t s_tmem,
 // starved by FMA-heavy neighbours.
 constexpr uint32_t kEmuMask = 0x88u;  // pairs 3 and 7 of each group of 8 (measured best of 0, 1/8, 2/8)
 
-// p = 2^(s * sl2 + nmu) for 32 pairs; the packed bf16 values go to TMEM at p_taddr in
-// two 16-column stores (so fewer of them are held in registers), (a0 + a1) gets the
+// p = 2^(s * sl2 + nmu) for 32 pairs, packed to bf16 pairs in P; (a0 + a1) gets the
 // fp32 sum.
 template <uint32_t MASK>
-__device__ __forceinline__ void exp_pairs(const float (&s)[64], float sl2, float nmu, uint32_t p_taddr, float& a0,
+__device__ __forceinline__ void exp_pairs(const float (&s)[64], float sl2, float nmu, uint32_t (&P)[32], float& a0,
                                           float& a1) {
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    uint32_t P[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int i = 16 * half + k;
-      float y0, y1, p0, p1;
-      fma2(y0, y1, s[2 * i], s[2 * i + 1], sl2, sl2, nmu, nmu);
-      if ((MASK >> (i & 7)) & 1u) {
-        exp2_fma2(p0, p1, y0, y1);
-      } else {
-        p0 = ex2(y0);
-        p1 = ex2(y1);
-      }
-      add2(a0, a1, p0, p1);
-      P[k] = pack_bf16x2(p0, p1);
+  for (int i = 0; i < 32; ++i) {
+    float y0, y1, p0, p1;
+    fma2(y0, y1, s[2 * i], s[2 * i + 1], sl2, sl2, nmu, nmu);
+    if ((MASK >> (i & 7)) & 1u) {
+      exp2_fma2(p0, p1, y0, y1);
+    } else {
+      p0 = ex2(y0);
+      p1 = ex2(y1);
     }
-    tmem_st16(p_taddr + 16 * half, P);
+    add2(a0, a1, p0, p1);
+    P[i] = pack_bf16x2(p0, p1);
   }
 }
 
-// Softmax over this thread's 64 columns of one row.  Returns the factor for the row's O.
-//
-// The exchange barrier also ORs `stop` over both halves, so that they leave the block
-// loop at the same block (a half that left alone would hang the other on the barrier).
-__device__ __forceinline__ float softmax_half_step(uint32_t s_taddr, bool masked, int col_limit, int col_low,
-                                                   float sl2,
-                                                   float* xmax_mine, const float* xmax_other, int bar_id,
-                                                   float& m, float& l, bool& stop) {
+// Row r's 64 probabilities (keys 64h..64h+63 of the block) into chunk h of the P tile,
+// K-major with the 128-byte swizzle: 16-byte granule g of row r sits at g ^ (r % 8).
+// A warp's store covers 32 rows x 16 bytes; within each group of 8 rows the granules
+// land in distinct bank groups.
+__device__ __forceinline__ void store_p_row(uint32_t chunk, int r, const uint32_t (&P)[32]) {
+  const uint32_t row = chunk + (uint32_t)r * 128u;
+#pragma unroll
+  for (int g = 0; g < 8; ++g)
+    st_shared_v4(row + (uint32_t)((g ^ (r & 7)) << 4), P[4 * g], P[4 * g + 1], P[4 * g + 2], P[4 * g + 3]);
+}
+
+// Loads this thread's 64 score columns of one block from TMEM, applies the mask and
+// returns their maximum (log2 units).
+template <bool LOW>
+__device__ __forceinline__ float load_scores(uint32_t s_taddr, bool masked, int col_limit, int col_low, float sl2,
+                                             float (&s)[64]) {
   uint32_t r[64];
   tmem_ld32(s_taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
   tmem_ld32(s_taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
   tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[0]));
   tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-  float s[64];
 #pragma unroll
   for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(r[c]);
   if (masked) {
 #pragma unroll
-    for (int c = 0; c < 64; ++c) s[c] = (c > col_limit || c < col_low) ? -INFINITY : s[c];
+    for (int c = 0; c < 64; ++c) s[c] = (c > col_limit || (LOW && c < col_low)) ? -INFINITY : s[c];
   }
   float x0 = max3(s[0], s[1], s[2]), x1 = max3(s[3], s[4], s[5]);
 #pragma unroll
@@ -438,26 +382,7 @@ __device__ __forceinline__ float softmax_half_step(uint32_t s_taddr, bool masked
     x0 = max3(x0, s[c], s[c + 1]);
     x1 = max3(x1, s[c + 2], s[c + 3]);
   }
-  float mx = max3(x0, x1, fmaxf(s[62], s[63])) * sl2;
-  *xmax_mine = mx;
-  stop = named_bar_sync_or(bar_id, 256, stop);
-  mx = fmaxf(mx, *xmax_other);
-
-  float alpha = 1.0f;
-  if (mx > m) {            // false while nothing is visible (mx = -inf)
-    alpha = ex2(m - mx);   // 0 when m = -inf
-    m = mx;
-  }
-  const float nmu = (m == -INFINITY) ? 0.0f : -m;
-
-  float a0 = 0.f, a1 = 0.f;
-  if (masked) {
-    exp_pairs<0u>(s, sl2, nmu, s_taddr, a0, a1);  // -inf entries: the exp unit returns exact zeros
-  } else {
-    exp_pairs<kEmuMask>(s, sl2, nmu, s_taddr, a0, a1);
-  }
-  l = l * alpha + (a0 + a1);
-  return alpha;
+  return max3(x0, x1, fmaxf(s[62], s[63])) * sl2;
 }
 
 template <int NC>
@@ -516,16 +441,21 @@ __device__ __forceinline__ void store_cols(const FwdArgs& a, uint32_t o_taddr, b
   }
 }
 
-template <int D>
+// MASKS = false: causal or no mask only (window = 0, block_mask = null); that
+// instance carries none of the window and block-map logic.
+template <int D, bool MASKS>
 __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_constant__ FwdArgs a) {
   using C = PingPongCfg<D>;
   constexpr int BN = C::BN;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_pp[];
+  uint8_t* smem = smem_pp;
+  if (smem_u32(smem) & 1023u) {  // the layout has no slack to realign (uniform exit, nothing started)
+    if (threadIdx.x == 0) latch_status(ATTN_ERR_ALIGNMENT);
+    return;
+  }
   PingPongBars* bars = reinterpret_cast<PingPongBars*>(smem + C::OFF_BAR);
-  PingPongRed* red = reinterpret_cast<PingPongRed*>(smem + C::OFF_RED);
-  CtaPlan* splan = reinterpret_cast<CtaPlan*>(smem + C::OFF_PLAN);
-  VisitEntry* vlist = reinterpret_cast<VisitEntry*>(smem + C::OFF_PLAN + 64);
+  float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
+  uint32_t* bitmaps = reinterpret_cast<uint32_t*>(smem + C::OFF_BITS);
   volatile int* abort_flag = &bars->abort_flag;
 
   const int warp = threadIdx.x >> 5;
@@ -550,8 +480,8 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
       }
       b = rem / hp_n;
       const int h0 = 2 * (rem % hp_n);
-      tj[0] = make_tile<BN>(a, h0, qt * 128);
-      tj[1] = make_tile<BN>(a, h0 + 1, qt * 128);
+      tj[0] = make_tile<BN, MASKS>(a, h0, qt * 128);
+      tj[1] = make_tile<BN, MASKS>(a, h0 + 1, qt * 128);
     } else {
       const int nqp = (a.n_qtiles + 1) / 2;
       int qp, rem;
@@ -564,8 +494,8 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
       }
       b = rem / a.Hq;
       const int h = rem % a.Hq;
-      tj[0] = make_tile<BN>(a, h, (2 * qp) * 128);
-      tj[1] = make_tile<BN>(a, h, (2 * qp + 1) * 128);
+      tj[0] = make_tile<BN, MASKS>(a, h, (2 * qp) * 128);
+      tj[1] = make_tile<BN, MASKS>(a, h, (2 * qp + 1) * 128);
     }
     kvh = tj[0].hq / a.group;
   }
@@ -574,6 +504,7 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->q_full[t], 1);
       mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->s_free[t], 8);
       mbar_init(&bars->p_full[t], 8);
       mbar_init(&bars->o_done[t], 1);
       mbar_init(&bars->o_final[t], 1);
@@ -590,24 +521,40 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
     tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 3 && a.block_mask != nullptr) build_list_plan<BN>(a, tj, 2, splan, vlist);
+  if (MASKS && a.block_mask != nullptr && (warp == 2 || warp == 3))
+    build_row_bitmap(a, tj[warp - 2], bitmaps + (warp - 2) * C::BITS_WORDS, C::BITS_WORDS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const CtaPlan plan = (a.block_mask != nullptr) ? *splan : range_plan(tj, 2);
-  const int nu = plan.nu;
   const uint32_t tmem = bars->tmem_base;
-  const uint32_t sQ[2] = {smem_u32(smem + C::OFF_Q), smem_u32(smem + C::OFF_Q + C::Q_BYTES)};
+  const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+  const uint32_t sP = smem_u32(smem + C::OFF_P);
   const uint32_t sKV = smem_u32(smem + C::OFF_KV);
+  const bool use_bits = MASKS && a.block_mask != nullptr;
+  const uint32_t* bits0 = use_bits ? bitmaps : nullptr;
+  const uint32_t* bits1 = use_bits ? bitmaps + C::BITS_WORDS : nullptr;
+
+  // visit walk: the union of both tiles' visited blocks, in increasing order
+  constexpr int kDone = 0x7fffffff;
+  auto tile_next = [&](int t, int kb) -> int {  // kDone if the tile visits nothing >= kb
+    const TileJob& j = t ? tj[1] : tj[0];
+    const int n = next_visit<BN>(t ? bits1 : bits0, j, kb);
+    return n < j.jhi ? n : kDone;
+  };
+  auto union_next = [&](int kb) -> int { return min(tile_next(0, kb), tile_next(1, kb)); };
+  auto visits = [&](int t, int kb) -> bool { return tile_visits<BN>(t ? bits1 : bits0, t ? tj[1] : tj[0], kb); };
 
   if (warp == 0) {
-    // ================= TMA producer: Q tiles, then K and V of every visited block
+    // ================= TMA producer: Q tiles, then K(u0), and per visited block u:
+    // K(next block), V(u)
     if (lane == 0) {
       tma_prefetch_map(&a.tm_q);
       tma_prefetch_map(&a.tm_k);
       tma_prefetch_map(&a.tm_v);
+      bool has[2];
       for (int t = 0; t < 2; ++t) {
-        if (plan.nv[t] == 0) continue;
+        has[t] = tile_next(t, 0) != kDone;
+        if (!has[t]) continue;
         mbar_arrive_expect_tx(&bars->q_full[t], C::Q_BYTES);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
@@ -615,87 +562,104 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
                       tj[t].q0, b * a.Hq + tj[t].hq);
       }
       const uint64_t pol = l2_policy_evict_last();
-      int it = 0;
-      bool ok = true;
-      for (int u = 0; u < nu && ok; ++u) {
-        const int kb = visit_at(plan, vlist, tj, u).kb;
-        for (int kv = 0; kv < 2 && ok; ++kv, ++it) {
-          const int st = it % C::NSTAGE;
-          const int use = it / C::NSTAGE;
-          if (use > 0 && !mbar_wait(&bars->kv_empty[st], (use - 1) & 1, abort_flag, a.timeout_ns)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&bars->kv_full[st], C::KV_BYTES);
-          const CUtensorMap* map = kv ? &a.tm_v : &a.tm_k;
+      int seq = 0;
+      auto push = [&](int kb, int kv) -> bool {
+        const int st = seq % C::NSTAGE;
+        const int use = seq / C::NSTAGE;
+        if (use > 0 && !mbar_wait(&bars->kv_empty[st], (use - 1) & 1, abort_flag, a.timeout_ns)) return false;
+        mbar_arrive_expect_tx(&bars->kv_full[st], C::KV_BYTES);
+        const CUtensorMap* map = kv ? &a.tm_v : &a.tm_k;
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d_hint(smem + C::OFF_KV + st * C::KV_BYTES + c * (BN * 128), map, &bars->kv_full[st],
-                             c * 64, kb * BN, b * a.Hkv + kvh, pol);
-        }
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d_hint(smem + C::OFF_KV + st * C::KV_BYTES + c * (BN * 128), map, &bars->kv_full[st], c * 64,
+                           kb * BN, b * a.Hkv + kvh, pol);
+        ++seq;
+        return true;
+      };
+      int kb = union_next(0);
+      bool ok = kb == kDone || push(kb, 0);
+      while (ok && kb != kDone) {
+        const int nk = union_next(kb + 1);
+        if (nk != kDone) ok = push(nk, 0);
+        if (ok) ok = push(kb, 1);
+        kb = nk;
       }
       // drain: every copy issued must have landed before the CTA may exit
       for (int t = 0; t < 2; ++t)
-        if (plan.nv[t] > 0) mbar_wait(&bars->q_full[t], 0, abort_flag, a.timeout_ns, false);
-      for (int st = 0; st < C::NSTAGE && st < it; ++st) {
-        const int last_use = (it - 1 - st) / C::NSTAGE;  // index of the last fill of stage st
+        if (has[t]) mbar_wait(&bars->q_full[t], 0, abort_flag, a.timeout_ns, false);
+      for (int st = 0; st < C::NSTAGE && st < seq; ++st) {
+        const int last_use = (seq - 1 - st) / C::NSTAGE;  // index of the last fill of stage st
         mbar_wait(&bars->kv_full[st], last_use & 1, abort_flag, a.timeout_ns, false);
       }
     }
   } else if (warp == 1) {
-    // ================= MMA issuer.  Order per visited block u:
-    //   P V_0(u), S_0(u+1), P V_1(u), S_1(u+1)
-    // (each only for the tiles that visit the block) so one tile's softmax overlaps the
-    // other tile's two MMAs.  S_t(u+1) overwrites the TMEM block that held P_t(u); it is
-    // issued after P V_t(u), and the tensor core executes one thread's MMAs in issue
-    // order.  Barrier phases count each tile's own visits.
-    if (lane == 0 && nu > 0) {
+    // ================= MMA issuer.  Consumes the ring in the producer's order.  S_t of a
+    // tile's next visit waits until the tile's softmax has read S_t (s_free); P V_t(u)
+    // waits for P_t (p_full).  Barrier phases count each tile's own visits.
+    int kb = union_next(0);
+    if (lane == 0 && kb != kDone) {
+      auto stage_of = [&](int seq) { return seq % C::NSTAGE; };
+      auto parity_of = [&](int seq) { return (uint32_t)((seq / C::NSTAGE) & 1); };
       bool ok = true;
       for (int t = 0; t < 2 && ok; ++t)
-        if (plan.nv[t] > 0) ok = mbar_wait(&bars->q_full[t], 0, abort_flag, a.timeout_ns);
-      auto stage_of = [&](int it) { return it % C::NSTAGE; };
-      auto parity_of = [&](int it) { return (uint32_t)((it / C::NSTAGE) & 1); };
-      int cnt[2] = {0, 0};  // visits of each tile issued so far (P V side)
-      Visit cur = visit_at(plan, vlist, tj, 0);
+        if (tile_next(t, 0) != kDone) ok = mbar_wait(&bars->q_full[t], 0, abort_flag, a.timeout_ns);
+      int seq = 0;
+      int nqk[2] = {0, 0}, npv[2] = {0, 0};
       if (ok) ok = mbar_wait(&bars->kv_full[stage_of(0)], parity_of(0), abort_flag, a.timeout_ns);
       if (ok) {
         tc_fence_after();
+#pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (!(cur.part >> t & 1)) continue;
-          issue_qk<D, BN>(tmem + (t ? C::COL_S1 : C::COL_S0), sQ[t], sKV + stage_of(0) * C::KV_BYTES);
+          if (!visits(t, kb)) continue;
+          issue_qk<D, BN>(tmem + (t ? C::COL_S1 : C::COL_S0), sQ + t * C::Q_BYTES, sKV + stage_of(0) * C::KV_BYTES);
           tc_commit(&bars->s_full[t]);
+          ++nqk[t];
         }
         tc_commit(&bars->kv_empty[stage_of(0)]);
+        seq = 1;
       }
-      for (int u = 0; u < nu && ok; ++u) {
-        const int itV = 2 * u + 1, itK = 2 * u + 2;
-        const bool more = u + 1 < nu;
-        const Visit nxt = more ? visit_at(plan, vlist, tj, u + 1) : Visit{0, 0};
-        if (!mbar_wait(&bars->kv_full[stage_of(itV)], parity_of(itV), abort_flag, a.timeout_ns)) break;
-        if (more && !mbar_wait(&bars->kv_full[stage_of(itK)], parity_of(itK), abort_flag, a.timeout_ns)) break;
-        const uint32_t sV = sKV + stage_of(itV) * C::KV_BYTES;
-        for (int t = 0; t < 2; ++t) {
-          const uint32_t colS = t ? C::COL_S1 : C::COL_S0;
-          const uint32_t colO = t ? C::COL_O1 : C::COL_O0;
-          if (cur.part >> t & 1) {
-            if (!mbar_wait(&bars->p_full[t], cnt[t] & 1, abort_flag, a.timeout_ns)) {
+      while (ok && kb != kDone) {
+        const int nk = union_next(kb + 1);
+        if (nk != kDone) {
+          // S_t(nk) = Q_t K(nk)^T for the tiles that visit nk
+          if (!mbar_wait(&bars->kv_full[stage_of(seq)], parity_of(seq), abort_flag, a.timeout_ns)) break;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (!ok || !visits(t, nk)) continue;
+            if (nqk[t] > 0 && !mbar_wait(&bars->s_free[t], (nqk[t] - 1) & 1, abort_flag, a.timeout_ns)) {
               ok = false;
-              break;
+              continue;
             }
             tc_fence_after();
-            issue_pv_split<D, BN>(tmem + colO, tmem + colS, sV, cnt[t] > 0);
-            tc_commit(&bars->o_done[t]);
-            if (++cnt[t] == plan.nv[t]) tc_commit(&bars->o_final[t]);
-          }
-          if (t == 1) tc_commit(&bars->kv_empty[stage_of(itV)]);
-          if (more && (nxt.part >> t & 1)) {
-            issue_qk<D, BN>(tmem + colS, sQ[t], sKV + stage_of(itK) * C::KV_BYTES);
+            issue_qk<D, BN>(tmem + (t ? C::COL_S1 : C::COL_S0), sQ + t * C::Q_BYTES,
+                            sKV + stage_of(seq) * C::KV_BYTES);
             tc_commit(&bars->s_full[t]);
+            ++nqk[t];
           }
+          if (!ok) break;
+          tc_commit(&bars->kv_empty[stage_of(seq)]);
+          ++seq;
+        }
+        // O_t += P_t(kb) V(kb)
+        if (!mbar_wait(&bars->kv_full[stage_of(seq)], parity_of(seq), abort_flag, a.timeout_ns)) break;
+        const uint32_t sV = sKV + stage_of(seq) * C::KV_BYTES;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!ok || !visits(t, kb)) continue;
+          if (!mbar_wait(&bars->p_full[t], npv[t] & 1, abort_flag, a.timeout_ns)) {
+            ok = false;
+            continue;
+          }
+          tc_fence_after();
+          issue_pv_ss<D, BN>(tmem + (t ? C::COL_O1 : C::COL_O0), sP + t * C::P_BYTES, sV, npv[t] > 0);
+          tc_commit(&bars->o_done[t]);
+          ++npv[t];
+          if (tile_next(t, kb + 1) == kDone) tc_commit(&bars->o_final[t]);  // the tile's last visit
         }
         if (!ok) break;
-        if (more) tc_commit(&bars->kv_empty[stage_of(itK)]);
-        cur = nxt;
+        tc_commit(&bars->kv_empty[stage_of(seq)]);
+        ++seq;
+        kb = nk;
       }
       // every MMA must be finished before TMEM is released
       tc_commit(&bars->drain);
@@ -708,63 +672,85 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
     const int h = (sw >> 2) & 1;
     const int quad = warp & 3;       // TMEM lane quadrant this warp may access
     const int r = quad * 32 + lane;  // row within the tile
-    const TileJob& job = tj[t];
+    const TileJob job = t ? tj[1] : tj[0];  // selects, not a dynamic index (no local memory)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t s_addr = tmem + lane_off + (t ? C::COL_S1 : C::COL_S0) + 64 * h;
     const uint32_t o_addr = tmem + lane_off + (t ? C::COL_O1 : C::COL_O0) + (D / 2) * h;
+    const uint32_t p_chunk = sP + t * C::P_BYTES + h * (C::P_BYTES / 2);
+    float* xmax_mine = xmax + (t * 2 + h) * 128 + r;
+    const float* xmax_other = xmax + (t * 2 + (h ^ 1)) * 128 + r;
     const int q = job.q0 + r;
     const int khi = row_key_limit(a, q) - 64 * h;  // limits relative to this half's first column
-    const int klo = row_key_low(a, q) - 64 * h;
+    const int klo = MASKS ? row_key_low(a, q) - 64 * h : 0;
     const int bar_id = 1 + t;
-    const int nv = plan.nv[t];
     float m = -INFINITY, l = 0.f;
-    bool ok = true;
     bool fail = false;  // a wait of this warp gave up; decided jointly at the next exchange
-    const bool use_list = plan.use_list != 0;
-    const int jlo = job.jlo;
-    int u = 0;  // list cursor
-    for (int k = 0; k < nv; ++k) {
-      int kb = jlo + k;  // range plan: the tile's blocks are contiguous
-      if (use_list) {
-        while (!(vlist[u].part >> t & 1)) ++u;
-        kb = vlist[u++].kb;
-      }
+    int k = 0;          // this tile's visits so far
+    for (int kb = tile_next(t, 0); kb != kDone; kb = tile_next(t, kb + 1), ++k) {
       // both halves reach the exchange barrier of every visit; an abort is decided
       // jointly there
       bool stop = fail || !mbar_wait(&bars->s_full[t], k & 1, abort_flag, a.timeout_ns) || *abort_flag;
       tc_fence_after();
-      const bool masked = block_needs_mask<BN>(a, job, kb);
-      const float alpha = softmax_half_step(s_addr, masked, khi - kb * BN, klo - kb * BN, a.scale_log2,
-                                            &red->xmax[t][k & 1][h][r], &red->xmax[t][k & 1][h ^ 1][r], bar_id,
-                                            m, l, stop);
+      float s[64];
+      const bool masked = block_needs_mask<BN, MASKS>(a, job, kb);
+      float mx = load_scores<MASKS>(s_addr, masked, khi - kb * BN, klo - kb * BN, a.scale_log2, s);
+      // The exchange slot is single-buffered: a half writes it again only after
+      // s_full of its next visit, which follows the MMA's wait for s_free of this visit
+      // from all 8 warps, which each give after reading the other half's value.
+      *xmax_mine = mx;
+      stop = named_bar_sync_or(bar_id, 256, stop);
+      mx = fmaxf(mx, *xmax_other);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->s_free[t]);
       if (stop) {
         fail = true;
         break;
       }
-      if (__any_sync(0xffffffffu, alpha != 1.0f) && k > 0) {
-        // O holds P V of earlier visits: wait for the last of those MMAs, then rescale
-        if (mbar_wait(&bars->o_done[t], (k - 1) & 1, abort_flag, a.timeout_ns)) {
-          tc_fence_after();
-          rescale_cols<D / 2>(o_addr, alpha);
-        } else {
-          fail = true;
-        }
+      float alpha = 1.0f;
+      if (mx > m) {           // false while nothing is visible (mx = -inf)
+        alpha = ex2(m - mx);  // 0 when m = -inf
+        m = mx;
       }
-      tmem_st_wait();
+      const float nmu = (m == -INFINITY) ? 0.0f : -m;
+      uint32_t P[32];
+      float a0 = 0.f, a1 = 0.f;
+      if (masked) {
+        exp_pairs<0u>(s, a.scale_log2, nmu, P, a0, a1);  // -inf entries: the exp unit returns exact zeros
+      } else {
+        exp_pairs<kEmuMask>(s, a.scale_log2, nmu, P, a0, a1);
+      }
+      l = l * alpha + (a0 + a1);
+      // P V of the previous visit must be done: it reads P_t, and O_t may be rescaled.
+      // (Warp-uniform decision: the stores and TMEM accesses below are per warp.)
+      if (!__all_sync(0xffffffffu, k == 0 || mbar_wait(&bars->o_done[t], (k - 1) & 1, abort_flag, a.timeout_ns))) {
+        fail = true;
+        continue;  // no P this visit: the MMA's wait gives up as well
+      }
+      store_p_row(p_chunk, r, P);
+      fence_proxy_async_smem();
+      if (k > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+        tc_fence_after();
+        rescale_cols<D / 2>(o_addr, alpha);
+        tmem_st_wait();
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full[t]);
     }
-    ok = !fail;
-    const bool have_o = nv > 0;
+    bool ok = !fail;
+    const bool have_o = k > 0;
     if (ok && have_o) {
       ok = mbar_wait(&bars->o_final[t], 0, abort_flag, a.timeout_ns);
       tc_fence_after();
     }
+    ok = __all_sync(0xffffffffu, ok);  // the TMEM loads of the epilogue are per warp
     // combine the two halves' row sums (same reference maximum, same rescale history)
-    red->sums[t][h][r] = l;
+    // through the tile's P buffer, which the last P V no longer reads
+    float* sums = reinterpret_cast<float*>(smem + C::OFF_P + t * C::P_BYTES);
+    sums[h * 128 + r] = l;
     named_bar_sync(bar_id, 256);
-    l += red->sums[t][h ^ 1][r];
+    l += sums[(h ^ 1) * 128 + r];
     if (ok) {
       const bool valid = r < job.rows;
       const size_t row = ((size_t)b * a.Hq + job.hq) * (size_t)a.Nq + (size_t)(valid ? q : 0);
@@ -794,6 +780,7 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
 // Returns the factor for the row's O.
 constexpr float kStaleMaxSlack = 8.0f;  // log2 units
 
+template <bool LOW>
 __device__ __forceinline__ float softmax_row64_step(uint32_t s_taddr, bool masked, int col_limit, int col_low,
                                                     float sl2, float& m, float& l, float& lr) {
   uint32_t r[64];
@@ -806,7 +793,7 @@ __device__ __forceinline__ float softmax_row64_step(uint32_t s_taddr, bool maske
   for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(r[c]);
   if (masked) {
 #pragma unroll
-    for (int c = 0; c < 64; ++c) s[c] = (c > col_limit || c < col_low) ? -INFINITY : s[c];
+    for (int c = 0; c < 64; ++c) s[c] = (c > col_limit || (LOW && c < col_low)) ? -INFINITY : s[c];
   }
   float x0 = max3(s[0], s[1], s[2]), x1 = max3(s[3], s[4], s[5]);
 #pragma unroll
@@ -875,23 +862,7 @@ struct SingleBars {
   uint32_t visible[32];  // block-sparse map row of the tile: bit mb = 128-key block mb
 };
 
-// Smallest block >= kb the tile visits (t.jhi if none).  bits: the tile's row of the
-// block-sparse map as a bitmap, or null when there is none.
-template <int BN>
-__device__ __forceinline__ int next_visit(const uint32_t* bits, const TileJob& t, int kb) {
-  if (kb < t.jlo) kb = t.jlo;
-  if (bits == nullptr) return kb < t.jhi ? kb : t.jhi;
-  while (kb < t.jhi) {
-    const int mb = kb * BN / kMaskBlock;
-    const uint32_t w = bits[mb >> 5] >> (mb & 31);
-    if (w & 1u) return kb;
-    const int skip = w ? __ffs(w) - 1 : 32 - (mb & 31);  // to the next set bit, or the next word
-    kb = (mb + skip) * (kMaskBlock / BN);
-  }
-  return t.jhi;
-}
-
-template <int D>
+template <int D, bool MASKS>
 __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_constant__ FwdArgs a) {
   using C = SingleCfg<D>;
   constexpr int BN = C::BN;
@@ -911,7 +882,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
     const int rem = a.causal ? u % per_level : u / a.n_qtiles;
     b = rem / a.Hq;
     hq = rem % a.Hq;
-    job = make_tile<BN>(a, hq, qt * 128);
+    job = make_tile<BN, MASKS>(a, hq, qt * 128);
   }
   const int kvh = hq / a.group;
 
@@ -935,22 +906,14 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
     tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 2 && a.block_mask != nullptr) {
-    // bitmap of the tile's map row (the host bounds nkt by 32 x 32)
-    const uint8_t* row = a.block_mask + (size_t)(job.q0 / kMaskBlock) * a.nkt;
-    for (int i = 0; i < 32; ++i) {
-      const int mb = 32 * i + lane;
-      const uint32_t w = __ballot_sync(0xffffffffu, mb < a.nkt && __ldg(&row[mb]) != 0);
-      if (lane == 0) bars->visible[i] = w;
-    }
-  }
+  if (MASKS && warp == 2 && a.block_mask != nullptr) build_row_bitmap(a, job, bars->visible, 32);  // nkt <= 1024
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const uint32_t sQ = smem_u32(smem + C::OFF_Q);
   const uint32_t sKV = smem_u32(smem + C::OFF_KV);
-  const uint32_t* bits = (a.block_mask != nullptr) ? bars->visible : nullptr;
+  const uint32_t* bits = (MASKS && a.block_mask != nullptr) ? bars->visible : nullptr;
   const int kb0 = next_visit<BN>(bits, job, job.jlo);  // first visited block
   const bool any = job.rows > 0 && kb0 < job.jhi;
 
@@ -1039,24 +1002,24 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
     const uint32_t o_addr = tmem + lane_off + C::COL_O;
     const int q = job.q0 + r;
     const int khi = row_key_limit(a, q);
-    const int klo = row_key_low(a, q);
+    const int klo = MASKS ? row_key_low(a, q) : 0;
     float m = -INFINITY, l = 0.f, lr = 0.f;
     bool ok = true;
     int j = 0;  // visits so far
     for (int kb = any ? kb0 : job.jhi; kb < job.jhi; kb = next_visit<BN>(bits, job, kb + 1), ++j) {
-      if (!mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag, a.timeout_ns)) {
-        ok = false;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag, a.timeout_ns))) {
+        ok = false;  // warp-uniform: the TMEM accesses are per warp
         break;
       }
       tc_fence_after();
       const uint32_t s_addr = tmem + lane_off + ((j & 1) ? C::COL_S1 : C::COL_S0);
-      const bool masked = block_needs_mask<BN>(a, job, kb);
+      const bool masked = block_needs_mask<BN, MASKS>(a, job, kb);
       const float alpha =
-          softmax_row64_step(s_addr, masked, khi - kb * BN, klo - kb * BN, a.scale_log2, m, l, lr);
+          softmax_row64_step<MASKS>(s_addr, masked, khi - kb * BN, klo - kb * BN, a.scale_log2, m, l, lr);
       if (__any_sync(0xffffffffu, alpha != 1.0f) && j > 0) {
         // P V(j-2) finished before S(j) (issued after it), so o_done is in phase j-1 or
         // later and its parity names P V(j-1) without ambiguity
-        if (!mbar_wait(&bars->o_done, (j - 1) & 1, abort_flag, a.timeout_ns)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done, (j - 1) & 1, abort_flag, a.timeout_ns))) {
           ok = false;
           break;
         }
@@ -1075,6 +1038,7 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
       ok = mbar_wait(&bars->o_final, 0, abort_flag, a.timeout_ns);
       tc_fence_after();
     }
+    ok = __all_sync(0xffffffffu, ok);
     if (ok) store_row<D>(a, o_addr, have_o, r < job.rows, b, hq, q, m, l, lr);
   }
 
