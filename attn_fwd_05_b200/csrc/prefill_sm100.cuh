@@ -255,7 +255,9 @@ __device__ __forceinline__ void store_row(const FwdArgs& a, uint32_t o_taddr, bo
 //
 // Warp roles (640 threads): warp 0 issues TMA loads, warp 1 issues the MMAs, warps 2-3
 // turn a block-sparse map into per-tile bitmaps (else idle), warps 4-19 are four
-// softmax warpgroups: tile t, column half h handled by warpgroup 1 + 2t + h.  Each
+// softmax warpgroups: tile t, column half h handled by warpgroup 1 + 2t + h.  (The
+// register file is split between the four schedulers, 16K registers each; with five
+// warps on each, 96 registers a thread is the most a launch can have.)  Each
 // softmax thread owns one query row of its tile and 64 of the 128 score columns of a
 // block; the two halves of a row exchange their block maxima through shared memory,
 // so both apply the same reference.
@@ -319,6 +321,25 @@ __device__ __forceinline__ void issue_pv_ss(uint32_t o_tmem, uint32_t sP, uint32
     const uint64_t db = db0 + (uint64_t)((kk * (16 * 128)) >> 4);
     mma_ss(o_tmem, da, db, idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
+}
+
+// The same two products with descriptors as word pairs (the pair kernel's MMA warp).
+template <int D, int BN>
+__device__ __forceinline__ void issue_qk_w(uint32_t s_tmem, Desc q, Desc k) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, BN, 0, 0);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk)
+    mma_ss_w(s_tmem, q.lo + (uint32_t)((((kk >> 2) * (128 * 128)) + (kk & 3) * 32) >> 4), q.hi,
+             k.lo + (uint32_t)((((kk >> 2) * (BN * 128)) + (kk & 3) * 32) >> 4), k.hi, idesc, kk > 0 ? 1u : 0u);
+}
+
+template <int D, int BN>
+__device__ __forceinline__ void issue_pv_w(uint32_t o_tmem, Desc p, Desc v, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk)
+    mma_ss_w(o_tmem, p.lo + (uint32_t)((((kk >> 2) * (128 * 128)) + (kk & 3) * 32) >> 4), p.hi,
+             v.lo + (uint32_t)((kk * (16 * 128)) >> 4), v.hi, idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // A quarter of the probability pairs (kEmuMask) is computed on the FMA pipe (exp2_fma2)
@@ -522,7 +543,7 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
     tmem_relinquish();
   }
   if (MASKS && a.block_mask != nullptr && (warp == 2 || warp == 3))
-    build_row_bitmap(a, tj[warp - 2], bitmaps + (warp - 2) * C::BITS_WORDS, C::BITS_WORDS);
+    build_row_bitmap(a, warp == 3 ? tj[1] : tj[0], bitmaps + (warp - 2) * C::BITS_WORDS, C::BITS_WORDS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -596,73 +617,102 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
     // ================= MMA issuer.  Consumes the ring in the producer's order.  S_t of a
     // tile's next visit waits until the tile's softmax has read S_t (s_free); P V_t(u)
     // waits for P_t (p_full).  Barrier phases count each tile's own visits.
+    // The whole warp runs this loop (waits, descriptors, bookkeeping are warp-uniform)
+    // and one elected lane issues the MMAs and commits: the issuing thread shares its
+    // scheduler with busy softmax warps, so each MMA should cost it few instructions.
     int kb = union_next(0);
-    if (lane == 0 && kb != kDone) {
+    if (kb != kDone) {
       auto stage_of = [&](int seq) { return seq % C::NSTAGE; };
       auto parity_of = [&](int seq) { return (uint32_t)((seq / C::NSTAGE) & 1); };
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.timeout_ns));
+      };
+      const Desc dq[2] = {desc_sw128(sQ, 16, 1024), desc_sw128(sQ + C::Q_BYTES, 16, 1024)};
+      const Desc dp[2] = {desc_sw128(sP, 16, 1024), desc_sw128(sP + C::P_BYTES, 16, 1024)};
+      const Desc dk0 = desc_sw128(sKV, 16, 1024);
+      const Desc dv0 = desc_sw128(sKV, BN * 128, 1024);
+      auto kdesc = [&](int seq) { return Desc{dk0.lo + (uint32_t)(stage_of(seq) * (C::KV_BYTES >> 4)), dk0.hi}; };
+      auto vdesc = [&](int seq) { return Desc{dv0.lo + (uint32_t)(stage_of(seq) * (C::KV_BYTES >> 4)), dv0.hi}; };
       bool ok = true;
       for (int t = 0; t < 2 && ok; ++t)
-        if (tile_next(t, 0) != kDone) ok = mbar_wait(&bars->q_full[t], 0, abort_flag, a.timeout_ns);
+        if (tile_next(t, 0) != kDone) ok = wait_all(&bars->q_full[t], 0);
       int seq = 0;
       int nqk[2] = {0, 0}, npv[2] = {0, 0};
-      if (ok) ok = mbar_wait(&bars->kv_full[stage_of(0)], parity_of(0), abort_flag, a.timeout_ns);
+      if (ok) ok = wait_all(&bars->kv_full[stage_of(0)], parity_of(0));
       if (ok) {
-        tc_fence_after();
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (!visits(t, kb)) continue;
-          issue_qk<D, BN>(tmem + (t ? C::COL_S1 : C::COL_S0), sQ + t * C::Q_BYTES, sKV + stage_of(0) * C::KV_BYTES);
-          tc_commit(&bars->s_full[t]);
-          ++nqk[t];
+        const bool v0 = visits(0, kb), v1 = visits(1, kb);
+        if (elect_one()) {
+          tc_fence_after();
+          if (v0) {
+            issue_qk_w<D, BN>(tmem + C::COL_S0, dq[0], kdesc(0));
+            tc_commit(&bars->s_full[0]);
+          }
+          if (v1) {
+            issue_qk_w<D, BN>(tmem + C::COL_S1, dq[1], kdesc(0));
+            tc_commit(&bars->s_full[1]);
+          }
+          tc_commit(&bars->kv_empty[stage_of(0)]);
         }
-        tc_commit(&bars->kv_empty[stage_of(0)]);
+        __syncwarp();
+        nqk[0] += v0;
+        nqk[1] += v1;
         seq = 1;
       }
       while (ok && kb != kDone) {
         const int nk = union_next(kb + 1);
         if (nk != kDone) {
           // S_t(nk) = Q_t K(nk)^T for the tiles that visit nk
-          if (!mbar_wait(&bars->kv_full[stage_of(seq)], parity_of(seq), abort_flag, a.timeout_ns)) break;
+          if (!wait_all(&bars->kv_full[stage_of(seq)], parity_of(seq))) break;
+          const Desc dk = kdesc(seq);
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             if (!ok || !visits(t, nk)) continue;
-            if (nqk[t] > 0 && !mbar_wait(&bars->s_free[t], (nqk[t] - 1) & 1, abort_flag, a.timeout_ns)) {
+            if (nqk[t] > 0 && !wait_all(&bars->s_free[t], (nqk[t] - 1) & 1)) {
               ok = false;
               continue;
             }
-            tc_fence_after();
-            issue_qk<D, BN>(tmem + (t ? C::COL_S1 : C::COL_S0), sQ + t * C::Q_BYTES,
-                            sKV + stage_of(seq) * C::KV_BYTES);
-            tc_commit(&bars->s_full[t]);
+            if (elect_one()) {
+              tc_fence_after();
+              issue_qk_w<D, BN>(tmem + (t ? C::COL_S1 : C::COL_S0), dq[t], dk);
+              tc_commit(&bars->s_full[t]);
+            }
+            __syncwarp();
             ++nqk[t];
           }
           if (!ok) break;
-          tc_commit(&bars->kv_empty[stage_of(seq)]);
+          if (elect_one()) tc_commit(&bars->kv_empty[stage_of(seq)]);
+          __syncwarp();
           ++seq;
         }
         // O_t += P_t(kb) V(kb)
-        if (!mbar_wait(&bars->kv_full[stage_of(seq)], parity_of(seq), abort_flag, a.timeout_ns)) break;
-        const uint32_t sV = sKV + stage_of(seq) * C::KV_BYTES;
+        if (!wait_all(&bars->kv_full[stage_of(seq)], parity_of(seq))) break;
+        const Desc dv = vdesc(seq);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           if (!ok || !visits(t, kb)) continue;
-          if (!mbar_wait(&bars->p_full[t], npv[t] & 1, abort_flag, a.timeout_ns)) {
+          if (!wait_all(&bars->p_full[t], npv[t] & 1)) {
             ok = false;
             continue;
           }
-          tc_fence_after();
-          issue_pv_ss<D, BN>(tmem + (t ? C::COL_O1 : C::COL_O0), sP + t * C::P_BYTES, sV, npv[t] > 0);
-          tc_commit(&bars->o_done[t]);
+          const bool last = tile_next(t, kb + 1) == kDone;  // the tile's last visit
+          if (elect_one()) {
+            tc_fence_after();
+            issue_pv_w<D, BN>(tmem + (t ? C::COL_O1 : C::COL_O0), dp[t], dv, npv[t] > 0);
+            tc_commit(&bars->o_done[t]);
+            if (last) tc_commit(&bars->o_final[t]);
+          }
+          __syncwarp();
           ++npv[t];
-          if (tile_next(t, kb + 1) == kDone) tc_commit(&bars->o_final[t]);  // the tile's last visit
         }
         if (!ok) break;
-        tc_commit(&bars->kv_empty[stage_of(seq)]);
+        if (elect_one()) tc_commit(&bars->kv_empty[stage_of(seq)]);
+        __syncwarp();
         ++seq;
         kb = nk;
       }
       // every MMA must be finished before TMEM is released
-      tc_commit(&bars->drain);
+      if (elect_one()) tc_commit(&bars->drain);
+      __syncwarp();
       mbar_wait(&bars->drain, 0, abort_flag, a.timeout_ns, false);
     }
   } else if (warp >= 4) {

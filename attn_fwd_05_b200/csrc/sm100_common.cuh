@@ -169,6 +169,34 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
       : "memory");
 }
 
+// Shared-memory descriptor as two 32-bit words.  The 14-bit start-address field sits at
+// the bottom of the low word and never carries (shared addresses are below 256 KB), so
+// operand offsets are plain 32-bit adds to `lo`.
+struct Desc {
+  uint32_t lo, hi;
+};
+
+// D(tmem) (+)= A(smem) * B(smem), descriptors as word pairs.
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo, uint32_t b_hi,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+      "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// True in exactly one lane of the (converged) warp: the lane that issues tensor-core
+// work for the warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 l;\n\telect.sync l|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // D(tmem) (+)= A(tmem) * B(smem)
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
@@ -196,6 +224,11 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   d |= (uint64_t)1u << 46;
   d |= (uint64_t)2u << 61;
   return d;
+}
+
+__device__ __forceinline__ Desc desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  const uint64_t d = smem_desc_sw128(saddr, lbo_bytes, sbo_bytes);
+  return Desc{(uint32_t)d, (uint32_t)(d >> 32)};
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B and an fp32
