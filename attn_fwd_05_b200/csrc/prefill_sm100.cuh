@@ -253,14 +253,12 @@ __device__ __forceinline__ void store_row(const FwdArgs& a, uint32_t o_taddr, bo
 // Kernel 1: two Q tiles per CTA (d = 64 or 128)
 // ====================================================================================
 //
-// Warp roles (640 threads): warp 0 issues TMA loads, warp 1 issues the MMAs, warps 2-3
-// turn a block-sparse map into per-tile bitmaps (else idle), warps 4-19 are four
-// softmax warpgroups: tile t, column half h handled by warpgroup 1 + 2t + h.  (The
-// register file is split between the four schedulers, 16K registers each; with five
-// warps on each, 96 registers a thread is the most a launch can have.)  Each
-// softmax thread owns one query row of its tile and 64 of the 128 score columns of a
-// block; the two halves of a row exchange their block maxima through shared memory,
-// so both apply the same reference.
+// Warp roles (384 threads): warp 0 issues TMA loads, warp 1 issues the MMAs, warps 2-3
+// turn a block-sparse map into per-tile bitmaps (else idle), warps 4-7 and 8-11 are the
+// softmax warpgroups of tiles 0 and 1.  Each softmax thread owns one query row of its
+// tile: all 128 scores of a block sit in its registers, so the row maximum needs no
+// exchange between threads.  Twelve warps leave three per scheduler and up to 168
+// registers a thread.
 //
 // P goes to shared memory (128-byte swizzled, K-major: the A operand of P V), not back
 // over S.  So S_t is free as soon as the softmax has read it into registers, and the
@@ -274,7 +272,7 @@ template <int D>
 struct PingPongCfg {
   static constexpr int BM = 128;
   static constexpr int BN = 128;
-  static constexpr int THREADS = 640;
+  static constexpr int THREADS = 384;
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int P_BYTES = BM * BN * 2;
   static constexpr int KV_BYTES = BN * D * 2;
@@ -282,8 +280,7 @@ struct PingPongCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_P = 2 * Q_BYTES;
   static constexpr int OFF_KV = OFF_P + 2 * P_BYTES;
-  static constexpr int OFF_XMAX = OFF_KV + NSTAGE * KV_BYTES;  // block maxima [tile][half][row]
-  static constexpr int OFF_BAR = OFF_XMAX + 2 * 2 * 128 * 4;
+  static constexpr int OFF_BAR = OFF_KV + NSTAGE * KV_BYTES;
   static constexpr int BAR_BYTES = 256;
   static constexpr int OFF_BITS = OFF_BAR + BAR_BYTES;  // block-sparse bitmaps [tile][64 words]
   static constexpr int BITS_WORDS = kMaxVisits / 32;
@@ -296,8 +293,8 @@ struct PingPongCfg {
 struct PingPongBars {
   uint64_t q_full[2];
   uint64_t s_full[2];   // S_t of the tile's next visit is in TMEM
-  uint64_t s_free[2];   // the tile's softmax has read S_t and exchanged its maxima (8 warps)
-  uint64_t p_full[2];   // P_t is in shared memory and O_t is rescaled (8 warps)
+  uint64_t s_free[2];   // the tile's softmax has read S_t (4 warps)
+  uint64_t p_full[2];   // P_t is in shared memory and O_t is rescaled (4 warps)
   uint64_t o_done[2];   // one phase per P V of the tile
   uint64_t o_final[2];  // one phase: the tile's last P V is done
   uint64_t drain;
@@ -350,13 +347,13 @@ __device__ __forceinline__ void issue_pv_w(uint32_t o_tmem, Desc p, Desc v, bool
 // starved by FMA-heavy neighbours.
 constexpr uint32_t kEmuMask = 0x88u;  // pairs 3 and 7 of each group of 8 (measured best of 0, 1/8, 2/8)
 
-// p = 2^(s * sl2 + nmu) for 32 pairs, packed to bf16 pairs in P; (a0 + a1) gets the
+// p = 2^(s * sl2 + nmu) for NP pairs, packed to bf16 pairs in P; (a0 + a1) gets the
 // fp32 sum.
-template <uint32_t MASK>
-__device__ __forceinline__ void exp_pairs(const float (&s)[64], float sl2, float nmu, uint32_t (&P)[32], float& a0,
-                                          float& a1) {
+template <uint32_t MASK, int NP>
+__device__ __forceinline__ void exp_pairs(const float (&s)[2 * NP], float sl2, float nmu, uint32_t (&P)[NP],
+                                          float& a0, float& a1) {
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NP; ++i) {
     float y0, y1, p0, p1;
     fma2(y0, y1, s[2 * i], s[2 * i + 1], sl2, sl2, nmu, nmu);
     if ((MASK >> (i & 7)) & 1u) {
@@ -370,40 +367,43 @@ __device__ __forceinline__ void exp_pairs(const float (&s)[64], float sl2, float
   }
 }
 
-// Row r's 64 probabilities (keys 64h..64h+63 of the block) into chunk h of the P tile,
-// K-major with the 128-byte swizzle: 16-byte granule g of row r sits at g ^ (r % 8).
-// A warp's store covers 32 rows x 16 bytes; within each group of 8 rows the granules
-// land in distinct bank groups.
-__device__ __forceinline__ void store_p_row(uint32_t chunk, int r, const uint32_t (&P)[32]) {
-  const uint32_t row = chunk + (uint32_t)r * 128u;
+// Row r's probabilities (NP pairs: keys 0 .. 2NP-1 of the block) into the P tile,
+// K-major with the 128-byte swizzle: keys 64c .. 64c+63 form chunk c (128 rows x 128
+// bytes), and 16-byte granule g of row r sits at g ^ (r % 8).  A warp's store covers
+// 32 rows x 16 bytes; within each group of 8 rows the granules land in distinct bank
+// groups.
+template <int NP>
+__device__ __forceinline__ void store_p_row(uint32_t p_tile, int r, const uint32_t (&P)[NP]) {
+  const uint32_t row = p_tile + (uint32_t)r * 128u;
 #pragma unroll
-  for (int g = 0; g < 8; ++g)
-    st_shared_v4(row + (uint32_t)((g ^ (r & 7)) << 4), P[4 * g], P[4 * g + 1], P[4 * g + 2], P[4 * g + 3]);
+  for (int g = 0; g < NP / 4; ++g)
+    st_shared_v4(row + (uint32_t)((g >> 3) * (128 * 128)) + (uint32_t)(((g & 7) ^ (r & 7)) << 4), P[4 * g],
+                 P[4 * g + 1], P[4 * g + 2], P[4 * g + 3]);
 }
 
-// Loads this thread's 64 score columns of one block from TMEM, applies the mask and
+// Loads this thread's NCOL score columns of one block from TMEM, applies the mask and
 // returns their maximum (log2 units).
-template <bool LOW>
+template <bool LOW, int NCOL>
 __device__ __forceinline__ float load_scores(uint32_t s_taddr, bool masked, int col_limit, int col_low, float sl2,
-                                             float (&s)[64]) {
-  uint32_t r[64];
-  tmem_ld32(s_taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-  tmem_ld32(s_taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-  tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-  tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+                                             float (&s)[NCOL]) {
+  uint32_t r[NCOL];
 #pragma unroll
-  for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(r[c]);
+  for (int c = 0; c < NCOL / 32; ++c) tmem_ld32(s_taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+#pragma unroll
+  for (int c = 0; c < NCOL / 32; ++c) tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+#pragma unroll
+  for (int c = 0; c < NCOL; ++c) s[c] = __uint_as_float(r[c]);
   if (masked) {
 #pragma unroll
-    for (int c = 0; c < 64; ++c) s[c] = (c > col_limit || (LOW && c < col_low)) ? -INFINITY : s[c];
+    for (int c = 0; c < NCOL; ++c) s[c] = (c > col_limit || (LOW && c < col_low)) ? -INFINITY : s[c];
   }
   float x0 = max3(s[0], s[1], s[2]), x1 = max3(s[3], s[4], s[5]);
 #pragma unroll
-  for (int c = 6; c < 62; c += 4) {
+  for (int c = 6; c < NCOL - 2; c += 4) {
     x0 = max3(x0, s[c], s[c + 1]);
     x1 = max3(x1, s[c + 2], s[c + 3]);
   }
-  return max3(x0, x1, fmaxf(s[62], s[63])) * sl2;
+  return max3(x0, x1, fmaxf(s[NCOL - 2], s[NCOL - 1])) * sl2;
 }
 
 template <int NC>
@@ -465,7 +465,7 @@ __device__ __forceinline__ void store_cols(const FwdArgs& a, uint32_t o_taddr, b
 // MASKS = false: causal or no mask only (window = 0, block_mask = null); that
 // instance carries none of the window and block-map logic.
 template <int D, bool MASKS>
-__global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_constant__ FwdArgs a) {
+__global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_constant__ FwdArgs a) {
   using C = PingPongCfg<D>;
   constexpr int BN = C::BN;
   extern __shared__ __align__(1024) uint8_t smem_pp[];
@@ -475,7 +475,6 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
     return;
   }
   PingPongBars* bars = reinterpret_cast<PingPongBars*>(smem + C::OFF_BAR);
-  float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
   uint32_t* bitmaps = reinterpret_cast<uint32_t*>(smem + C::OFF_BITS);
   volatile int* abort_flag = &bars->abort_flag;
 
@@ -525,8 +524,8 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->q_full[t], 1);
       mbar_init(&bars->s_full[t], 1);
-      mbar_init(&bars->s_free[t], 8);
-      mbar_init(&bars->p_full[t], 8);
+      mbar_init(&bars->s_free[t], 4);
+      mbar_init(&bars->p_full[t], 4);
       mbar_init(&bars->o_done[t], 1);
       mbar_init(&bars->o_final[t], 1);
     }
@@ -716,72 +715,60 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
       mbar_wait(&bars->drain, 0, abort_flag, a.timeout_ns, false);
     }
   } else if (warp >= 4) {
-    // ================= softmax: warpgroup 1 + 2t + h owns tile t, column half h
-    const int sw = warp - 4;
-    const int t = sw >> 3;
-    const int h = (sw >> 2) & 1;
+    // ================= softmax: warps 4 + 4t .. 7 + 4t own tile t, one row per thread
+    const int t = (warp - 4) >> 2;
     const int quad = warp & 3;       // TMEM lane quadrant this warp may access
     const int r = quad * 32 + lane;  // row within the tile
     const TileJob job = t ? tj[1] : tj[0];  // selects, not a dynamic index (no local memory)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t s_addr = tmem + lane_off + (t ? C::COL_S1 : C::COL_S0) + 64 * h;
-    const uint32_t o_addr = tmem + lane_off + (t ? C::COL_O1 : C::COL_O0) + (D / 2) * h;
-    const uint32_t p_chunk = sP + t * C::P_BYTES + h * (C::P_BYTES / 2);
-    float* xmax_mine = xmax + (t * 2 + h) * 128 + r;
-    const float* xmax_other = xmax + (t * 2 + (h ^ 1)) * 128 + r;
+    const uint32_t s_addr = tmem + lane_off + (t ? C::COL_S1 : C::COL_S0);
+    const uint32_t o_addr = tmem + lane_off + (t ? C::COL_O1 : C::COL_O0);
+    const uint32_t p_tile = sP + t * C::P_BYTES;
     const int q = job.q0 + r;
-    const int khi = row_key_limit(a, q) - 64 * h;  // limits relative to this half's first column
-    const int klo = MASKS ? row_key_low(a, q) - 64 * h : 0;
-    const int bar_id = 1 + t;
+    const int khi = row_key_limit(a, q);
+    const int klo = MASKS ? row_key_low(a, q) : 0;
     float m = -INFINITY, l = 0.f;
-    bool fail = false;  // a wait of this warp gave up; decided jointly at the next exchange
+    bool fail = false;  // a wait gave up (the warp decides as one)
     int k = 0;          // this tile's visits so far
     for (int kb = tile_next(t, 0); kb != kDone; kb = tile_next(t, kb + 1), ++k) {
-      // both halves reach the exchange barrier of every visit; an abort is decided
-      // jointly there
-      bool stop = fail || !mbar_wait(&bars->s_full[t], k & 1, abort_flag, a.timeout_ns) || *abort_flag;
-      tc_fence_after();
-      float s[64];
-      const bool masked = block_needs_mask<BN, MASKS>(a, job, kb);
-      float mx = load_scores<MASKS>(s_addr, masked, khi - kb * BN, klo - kb * BN, a.scale_log2, s);
-      // The exchange slot is single-buffered: a half writes it again only after
-      // s_full of its next visit, which follows the MMA's wait for s_free of this visit
-      // from all 8 warps, which each give after reading the other half's value.
-      *xmax_mine = mx;
-      stop = named_bar_sync_or(bar_id, 256, stop);
-      mx = fmaxf(mx, *xmax_other);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->s_free[t]);
-      if (stop) {
+      if (__any_sync(0xffffffffu, !mbar_wait(&bars->s_full[t], k & 1, abort_flag, a.timeout_ns) || *abort_flag)) {
         fail = true;
         break;
       }
+      tc_fence_after();
+      float s[BN];
+      const bool masked = block_needs_mask<BN, MASKS>(a, job, kb);
+      const float mx = load_scores<MASKS, BN>(s_addr, masked, khi - kb * BN, klo - kb * BN, a.scale_log2, s);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->s_free[t]);  // S_t may be overwritten
+      // exact running maximum: whenever it grows, O is rescaled before this block's P V,
+      // so the row's largest probability is exactly 1 and its bf16 rounding is exact
       float alpha = 1.0f;
       if (mx > m) {           // false while nothing is visible (mx = -inf)
         alpha = ex2(m - mx);  // 0 when m = -inf
         m = mx;
       }
       const float nmu = (m == -INFINITY) ? 0.0f : -m;
-      uint32_t P[32];
+      uint32_t P[BN / 2];
       float a0 = 0.f, a1 = 0.f;
-      if (masked) {
-        exp_pairs<0u>(s, a.scale_log2, nmu, P, a0, a1);  // -inf entries: the exp unit returns exact zeros
+      if (masked) {  // -inf entries: the exp unit returns exact zeros
+        exp_pairs<0u, BN / 2>(s, a.scale_log2, nmu, P, a0, a1);
       } else {
-        exp_pairs<kEmuMask>(s, a.scale_log2, nmu, P, a0, a1);
+        exp_pairs<kEmuMask, BN / 2>(s, a.scale_log2, nmu, P, a0, a1);
       }
       l = l * alpha + (a0 + a1);
       // P V of the previous visit must be done: it reads P_t, and O_t may be rescaled.
       // (Warp-uniform decision: the stores and TMEM accesses below are per warp.)
       if (!__all_sync(0xffffffffu, k == 0 || mbar_wait(&bars->o_done[t], (k - 1) & 1, abort_flag, a.timeout_ns))) {
         fail = true;
-        continue;  // no P this visit: the MMA's wait gives up as well
+        break;
       }
-      store_p_row(p_chunk, r, P);
+      store_p_row<BN / 2>(p_tile, r, P);
       fence_proxy_async_smem();
       if (k > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
         tc_fence_after();
-        rescale_cols<D / 2>(o_addr, alpha);
+        rescale_cols<D>(o_addr, alpha);
         tmem_st_wait();
       }
       tc_fence_before();
@@ -795,17 +782,11 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
       tc_fence_after();
     }
     ok = __all_sync(0xffffffffu, ok);  // the TMEM loads of the epilogue are per warp
-    // combine the two halves' row sums (same reference maximum, same rescale history)
-    // through the tile's P buffer, which the last P V no longer reads
-    float* sums = reinterpret_cast<float*>(smem + C::OFF_P + t * C::P_BYTES);
-    sums[h * 128 + r] = l;
-    named_bar_sync(bar_id, 256);
-    l += sums[(h ^ 1) * 128 + r];
     if (ok) {
       const bool valid = r < job.rows;
       const size_t row = ((size_t)b * a.Hq + job.hq) * (size_t)a.Nq + (size_t)(valid ? q : 0);
-      store_cols<D / 2>(a, o_addr, have_o, valid, row * D + (D / 2) * h, l);
-      if (h == 0 && valid && a.lse != nullptr) a.lse[row] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
+      store_cols<D>(a, o_addr, have_o, valid, row * D, l);
+      if (valid && a.lse != nullptr) a.lse[row] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
     }
   }
 
@@ -828,6 +809,7 @@ __global__ void __launch_bounds__(640, 1) attn_fwd_pingpong_kernel(const __grid_
 // the bf16-rounded P that multiply V, normalises O (the rounding of a dominant
 // probability cancels in the ratio); l, the fp32 sum, gives the log-sum-exp.
 // Returns the factor for the row's O.
+
 constexpr float kStaleMaxSlack = 8.0f;  // log2 units
 
 template <bool LOW>
