@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -107,7 +108,9 @@ attn_status launch_prefill(attn::FwdArgs& a, cudaStream_t st) {
     const long long units = a.pair_heads ? (long long)a.B * (a.Hq / 2) * a.n_qtiles : (long long)a.B * a.Hq * qp;
     if (units <= 0 || units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
     a.n_units = (int)units;
-    k<<<(unsigned)units, C::THREADS, C::SMEM, st>>>(a);
+    // persistent: one CTA per SM walks the units; with a block-sparse map, one unit per CTA
+    const long long grid = a.block_mask != nullptr ? units : std::min<long long>(units, sm_count());
+    k<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(a);
   } else {
     using C = attn::SingleCfg<D>;
     auto k = attn::attn_fwd_single_kernel<D, MASKS>;

@@ -292,6 +292,7 @@ struct PingPongCfg {
 
 struct PingPongBars {
   uint64_t q_full[2];
+  uint64_t q_empty[2];  // the unit's last S_t = Q_t K^T is done: Q_t may be reloaded
   uint64_t s_full[2];   // S_t of the tile's next visit is in TMEM
   uint64_t s_free[2];   // the tile's softmax has read S_t (4 warps)
   uint64_t p_full[2];   // P_t is in shared memory and O_t is rescaled (4 warps)
@@ -462,8 +463,53 @@ __device__ __forceinline__ void store_cols(const FwdArgs& a, uint32_t o_taddr, b
   }
 }
 
-// MASKS = false: causal or no mask only (window = 0, block_mask = null); that
-// instance carries none of the window and block-map logic.
+// Work unit u of the two-tile kernel: two 128-row Q tiles and the KV head they read.
+// Causal: heaviest q-tiles first (longest-processing-time order).  Otherwise all units
+// weigh about the same; consecutive units share a head so that the K/V tiles streamed at
+// the same time stay in L2.
+template <int BN, bool MASKS>
+__device__ __forceinline__ void unit_tiles(const FwdArgs& a, int u, int& b, int& kvh, TileJob (&tj)[2]) {
+  if (a.pair_heads) {
+    const int hp_n = a.Hq / 2;
+    int qt, rem;
+    if (a.causal) {
+      qt = a.n_qtiles - 1 - u / (a.B * hp_n);
+      rem = u % (a.B * hp_n);
+    } else {
+      qt = u % a.n_qtiles;
+      rem = u / a.n_qtiles;
+    }
+    b = rem / hp_n;
+    const int h0 = 2 * (rem % hp_n);
+    tj[0] = make_tile<BN, MASKS>(a, h0, qt * 128);
+    tj[1] = make_tile<BN, MASKS>(a, h0 + 1, qt * 128);
+  } else {
+    const int nqp = (a.n_qtiles + 1) / 2;
+    int qp, rem;
+    if (a.causal) {
+      qp = nqp - 1 - u / (a.B * a.Hq);
+      rem = u % (a.B * a.Hq);
+    } else {
+      qp = u % nqp;
+      rem = u / nqp;
+    }
+    b = rem / a.Hq;
+    const int h = rem % a.Hq;
+    tj[0] = make_tile<BN, MASKS>(a, h, (2 * qp) * 128);
+    tj[1] = make_tile<BN, MASKS>(a, h, (2 * qp + 1) * 128);
+  }
+  kvh = tj[0].hq / a.group;
+}
+
+// Persistent: in round r CTA c takes unit r G + c (r even) or r G + G - 1 - c (r odd),
+// G = gridDim.x.  Every role walks the same unit
+// sequence and every barrier keeps counting across units, so the next unit's Q and K
+// loads and its first S = Q K^T run while the current unit's last softmax step and
+// epilogue are still going.  With a block-sparse map each CTA takes exactly one unit
+// (the map row becomes bitmaps once, before the roles start).
+//
+// MASKS = false: causal or no mask only (window = 0, block_mask = null); that instance
+// carries none of the window and block-map logic.
 template <int D, bool MASKS>
 __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_constant__ FwdArgs a) {
   using C = PingPongCfg<D>;
@@ -480,49 +526,12 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- work unit.  Causal: heaviest q-tiles first (longest-processing-time order).
-  // Otherwise: all units weigh about the same; consecutive CTAs share a head so that the
-  // K/V tiles they all stream stay in L2.
-  int b, kvh;
-  TileJob tj[2];
-  {
-    const int u = blockIdx.x;
-    if (a.pair_heads) {
-      const int hp_n = a.Hq / 2;
-      int qt, rem;
-      if (a.causal) {
-        qt = a.n_qtiles - 1 - u / (a.B * hp_n);
-        rem = u % (a.B * hp_n);
-      } else {
-        qt = u % a.n_qtiles;
-        rem = u / a.n_qtiles;
-      }
-      b = rem / hp_n;
-      const int h0 = 2 * (rem % hp_n);
-      tj[0] = make_tile<BN, MASKS>(a, h0, qt * 128);
-      tj[1] = make_tile<BN, MASKS>(a, h0 + 1, qt * 128);
-    } else {
-      const int nqp = (a.n_qtiles + 1) / 2;
-      int qp, rem;
-      if (a.causal) {
-        qp = nqp - 1 - u / (a.B * a.Hq);
-        rem = u % (a.B * a.Hq);
-      } else {
-        qp = u % nqp;
-        rem = u / nqp;
-      }
-      b = rem / a.Hq;
-      const int h = rem % a.Hq;
-      tj[0] = make_tile<BN, MASKS>(a, h, (2 * qp) * 128);
-      tj[1] = make_tile<BN, MASKS>(a, h, (2 * qp + 1) * 128);
-    }
-    kvh = tj[0].hq / a.group;
-  }
+  const bool use_bits = MASKS && a.block_mask != nullptr;
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->q_full[t], 1);
+      mbar_init(&bars->q_empty[t], 1);
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->s_free[t], 4);
       mbar_init(&bars->p_full[t], 4);
@@ -541,8 +550,12 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
     tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (MASKS && a.block_mask != nullptr && (warp == 2 || warp == 3))
+  int b, kvh;
+  TileJob tj[2];
+  if (use_bits && (warp == 2 || warp == 3)) {  // one unit per CTA here (host launch)
+    unit_tiles<BN, MASKS>(a, blockIdx.x, b, kvh, tj);
     build_row_bitmap(a, warp == 3 ? tj[1] : tj[0], bitmaps + (warp - 2) * C::BITS_WORDS, C::BITS_WORDS);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -550,11 +563,10 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
   const uint32_t sQ = smem_u32(smem + C::OFF_Q);
   const uint32_t sP = smem_u32(smem + C::OFF_P);
   const uint32_t sKV = smem_u32(smem + C::OFF_KV);
-  const bool use_bits = MASKS && a.block_mask != nullptr;
   const uint32_t* bits0 = use_bits ? bitmaps : nullptr;
   const uint32_t* bits1 = use_bits ? bitmaps + C::BITS_WORDS : nullptr;
 
-  // visit walk: the union of both tiles' visited blocks, in increasing order
+  // visit walk of the current unit: the union of both tiles' visited blocks, in order
   constexpr int kDone = 0x7fffffff;
   auto tile_next = [&](int t, int kb) -> int {  // kDone if the tile visits nothing >= kb
     const TileJob& j = t ? tj[1] : tj[0];
@@ -563,26 +575,23 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
   };
   auto union_next = [&](int kb) -> int { return min(tile_next(0, kb), tile_next(1, kb)); };
   auto visits = [&](int t, int kb) -> bool { return tile_visits<BN>(t ? bits1 : bits0, t ? tj[1] : tj[0], kb); };
+  // unit of round rd: rounds alternate direction over the CTAs, so that with the units
+  // sorted heaviest first every CTA's total stays close to the mean
+  auto snake_unit = [&](int rd) -> int {
+    return rd * (int)gridDim.x + ((rd & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+  };
 
   if (warp == 0) {
-    // ================= TMA producer: Q tiles, then K(u0), and per visited block u:
+    // ================= TMA producer.  Per unit: the Q tiles (each once the previous
+    // unit's last S of that tile is done), then K(u0), and per visited block u:
     // K(next block), V(u)
     if (lane == 0) {
       tma_prefetch_map(&a.tm_q);
       tma_prefetch_map(&a.tm_k);
       tma_prefetch_map(&a.tm_v);
-      bool has[2];
-      for (int t = 0; t < 2; ++t) {
-        has[t] = tile_next(t, 0) != kDone;
-        if (!has[t]) continue;
-        mbar_arrive_expect_tx(&bars->q_full[t], C::Q_BYTES);
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + C::OFF_Q + t * C::Q_BYTES + c * (128 * 128), &a.tm_q, &bars->q_full[t], c * 64,
-                      tj[t].q0, b * a.Hq + tj[t].hq);
-      }
       const uint64_t pol = l2_policy_evict_last();
       int seq = 0;
+      int nql[2] = {0, 0};  // Q loads of each tile so far
       auto push = [&](int kb, int kv) -> bool {
         const int st = seq % C::NSTAGE;
         const int use = seq / C::NSTAGE;
@@ -596,17 +605,37 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
         ++seq;
         return true;
       };
-      int kb = union_next(0);
-      bool ok = kb == kDone || push(kb, 0);
-      while (ok && kb != kDone) {
-        const int nk = union_next(kb + 1);
-        if (nk != kDone) ok = push(nk, 0);
-        if (ok) ok = push(kb, 1);
-        kb = nk;
+      bool ok = true;
+      for (int rd = 0; rd * (int)gridDim.x < a.n_units && ok; ++rd) {
+        const int u = snake_unit(rd);
+        if (u >= a.n_units) continue;
+        unit_tiles<BN, MASKS>(a, u, b, kvh, tj);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (tile_next(t, 0) == kDone) continue;
+          if (nql[t] > 0 && !mbar_wait(&bars->q_empty[t], (nql[t] - 1) & 1, abort_flag, a.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars->q_full[t], C::Q_BYTES);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem + C::OFF_Q + t * C::Q_BYTES + c * (128 * 128), &a.tm_q, &bars->q_full[t], c * 64,
+                        tj[t].q0, b * a.Hq + tj[t].hq);
+          ++nql[t];
+        }
+        int kb = union_next(0);
+        if (ok && kb != kDone) ok = push(kb, 0);
+        while (ok && kb != kDone) {
+          const int nk = union_next(kb + 1);
+          if (nk != kDone) ok = push(nk, 0);
+          if (ok) ok = push(kb, 1);
+          kb = nk;
+        }
       }
-      // drain: every copy issued must have landed before the CTA may exit
+      // drain: every copy issued must have landed before the CTA may exit (a Q tile is
+      // reloaded only after the previous load was consumed, so only the last can fly)
       for (int t = 0; t < 2; ++t)
-        if (has[t]) mbar_wait(&bars->q_full[t], 0, abort_flag, a.timeout_ns, false);
+        if (nql[t] > 0) mbar_wait(&bars->q_full[t], (nql[t] - 1) & 1, abort_flag, a.timeout_ns, false);
       for (int st = 0; st < C::NSTAGE && st < seq; ++st) {
         const int last_use = (seq - 1 - st) / C::NSTAGE;  // index of the last fill of stage st
         mbar_wait(&bars->kv_full[st], last_use & 1, abort_flag, a.timeout_ns, false);
@@ -615,76 +644,71 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
   } else if (warp == 1) {
     // ================= MMA issuer.  Consumes the ring in the producer's order.  S_t of a
     // tile's next visit waits until the tile's softmax has read S_t (s_free); P V_t(u)
-    // waits for P_t (p_full).  Barrier phases count each tile's own visits.
+    // waits for P_t (p_full).  Barrier phases count each tile's visits over all units.
     // The whole warp runs this loop (waits, descriptors, bookkeeping are warp-uniform)
     // and one elected lane issues the MMAs and commits: the issuing thread shares its
     // scheduler with busy softmax warps, so each MMA should cost it few instructions.
-    int kb = union_next(0);
-    if (kb != kDone) {
-      auto stage_of = [&](int seq) { return seq % C::NSTAGE; };
-      auto parity_of = [&](int seq) { return (uint32_t)((seq / C::NSTAGE) & 1); };
-      auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.timeout_ns));
-      };
-      const Desc dq[2] = {desc_sw128(sQ, 16, 1024), desc_sw128(sQ + C::Q_BYTES, 16, 1024)};
-      const Desc dp[2] = {desc_sw128(sP, 16, 1024), desc_sw128(sP + C::P_BYTES, 16, 1024)};
-      const Desc dk0 = desc_sw128(sKV, 16, 1024);
-      const Desc dv0 = desc_sw128(sKV, BN * 128, 1024);
-      auto kdesc = [&](int seq) { return Desc{dk0.lo + (uint32_t)(stage_of(seq) * (C::KV_BYTES >> 4)), dk0.hi}; };
-      auto vdesc = [&](int seq) { return Desc{dv0.lo + (uint32_t)(stage_of(seq) * (C::KV_BYTES >> 4)), dv0.hi}; };
-      bool ok = true;
-      for (int t = 0; t < 2 && ok; ++t)
-        if (tile_next(t, 0) != kDone) ok = wait_all(&bars->q_full[t], 0);
-      int seq = 0;
-      int nqk[2] = {0, 0}, npv[2] = {0, 0};
-      if (ok) ok = wait_all(&bars->kv_full[stage_of(0)], parity_of(0));
-      if (ok) {
-        const bool v0 = visits(0, kb), v1 = visits(1, kb);
+    auto stage_of = [&](int seq) { return seq % C::NSTAGE; };
+    auto parity_of = [&](int seq) { return (uint32_t)((seq / C::NSTAGE) & 1); };
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.timeout_ns));
+    };
+    const Desc dq[2] = {desc_sw128(sQ, 16, 1024), desc_sw128(sQ + C::Q_BYTES, 16, 1024)};
+    const Desc dp[2] = {desc_sw128(sP, 16, 1024), desc_sw128(sP + C::P_BYTES, 16, 1024)};
+    const Desc dk0 = desc_sw128(sKV, 16, 1024);
+    const Desc dv0 = desc_sw128(sKV, BN * 128, 1024);
+    auto kdesc = [&](int seq) { return Desc{dk0.lo + (uint32_t)(stage_of(seq) * (C::KV_BYTES >> 4)), dk0.hi}; };
+    auto vdesc = [&](int seq) { return Desc{dv0.lo + (uint32_t)(stage_of(seq) * (C::KV_BYTES >> 4)), dv0.hi}; };
+    int seq = 0;
+    int nqk[2] = {0, 0}, npv[2] = {0, 0}, nql[2] = {0, 0};
+    bool ok = true;
+    // S_t(kb) = Q_t K(kb)^T for the tiles that visit kb; K(kb) is ring entry seq
+    auto issue_s = [&](int kb) -> bool {
+      if (!wait_all(&bars->kv_full[stage_of(seq)], parity_of(seq))) return false;
+      const Desc dk = kdesc(seq);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (!visits(t, kb)) continue;
+        if (nqk[t] > 0 && !wait_all(&bars->s_free[t], (nqk[t] - 1) & 1)) return false;
+        const bool last = tile_next(t, kb + 1) == kDone;  // the unit's last S of this tile
         if (elect_one()) {
           tc_fence_after();
-          if (v0) {
-            issue_qk_w<D, BN>(tmem + C::COL_S0, dq[0], kdesc(0));
-            tc_commit(&bars->s_full[0]);
-          }
-          if (v1) {
-            issue_qk_w<D, BN>(tmem + C::COL_S1, dq[1], kdesc(0));
-            tc_commit(&bars->s_full[1]);
-          }
-          tc_commit(&bars->kv_empty[stage_of(0)]);
+          issue_qk_w<D, BN>(tmem + (t ? C::COL_S1 : C::COL_S0), dq[t], dk);
+          tc_commit(&bars->s_full[t]);
+          if (last) tc_commit(&bars->q_empty[t]);
         }
         __syncwarp();
-        nqk[0] += v0;
-        nqk[1] += v1;
-        seq = 1;
+        ++nqk[t];
       }
+      if (elect_one()) tc_commit(&bars->kv_empty[stage_of(seq)]);
+      __syncwarp();
+      ++seq;
+      return true;
+    };
+    for (int rd = 0; rd * (int)gridDim.x < a.n_units && ok; ++rd) {
+      const int u = snake_unit(rd);
+      if (u >= a.n_units) continue;
+      unit_tiles<BN, MASKS>(a, u, b, kvh, tj);
+      int kb = union_next(0);
+      if (kb == kDone) continue;
+      int upv[2] = {0, 0};  // P V of each tile in this unit (the first one overwrites O_t)
+      for (int t = 0; t < 2 && ok; ++t) {
+        if (tile_next(t, 0) == kDone) continue;
+        ok = wait_all(&bars->q_full[t], nql[t] & 1);
+        ++nql[t];
+      }
+      if (ok) ok = issue_s(kb);
       while (ok && kb != kDone) {
         const int nk = union_next(kb + 1);
-        if (nk != kDone) {
-          // S_t(nk) = Q_t K(nk)^T for the tiles that visit nk
-          if (!wait_all(&bars->kv_full[stage_of(seq)], parity_of(seq))) break;
-          const Desc dk = kdesc(seq);
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (!ok || !visits(t, nk)) continue;
-            if (nqk[t] > 0 && !wait_all(&bars->s_free[t], (nqk[t] - 1) & 1)) {
-              ok = false;
-              continue;
-            }
-            if (elect_one()) {
-              tc_fence_after();
-              issue_qk_w<D, BN>(tmem + (t ? C::COL_S1 : C::COL_S0), dq[t], dk);
-              tc_commit(&bars->s_full[t]);
-            }
-            __syncwarp();
-            ++nqk[t];
-          }
-          if (!ok) break;
-          if (elect_one()) tc_commit(&bars->kv_empty[stage_of(seq)]);
-          __syncwarp();
-          ++seq;
+        if (nk != kDone && !issue_s(nk)) {
+          ok = false;
+          break;
         }
         // O_t += P_t(kb) V(kb)
-        if (!wait_all(&bars->kv_full[stage_of(seq)], parity_of(seq))) break;
+        if (!wait_all(&bars->kv_full[stage_of(seq)], parity_of(seq))) {
+          ok = false;
+          break;
+        }
         const Desc dv = vdesc(seq);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
@@ -693,15 +717,16 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
             ok = false;
             continue;
           }
-          const bool last = tile_next(t, kb + 1) == kDone;  // the tile's last visit
+          const bool last = tile_next(t, kb + 1) == kDone;  // the tile's last visit of the unit
           if (elect_one()) {
             tc_fence_after();
-            issue_pv_w<D, BN>(tmem + (t ? C::COL_O1 : C::COL_O0), dp[t], dv, npv[t] > 0);
+            issue_pv_w<D, BN>(tmem + (t ? C::COL_O1 : C::COL_O0), dp[t], dv, upv[t] > 0);
             tc_commit(&bars->o_done[t]);
             if (last) tc_commit(&bars->o_final[t]);
           }
           __syncwarp();
           ++npv[t];
+          ++upv[t];
         }
         if (!ok) break;
         if (elect_one()) tc_commit(&bars->kv_empty[stage_of(seq)]);
@@ -709,80 +734,95 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
         ++seq;
         kb = nk;
       }
-      // every MMA must be finished before TMEM is released
-      if (elect_one()) tc_commit(&bars->drain);
-      __syncwarp();
-      mbar_wait(&bars->drain, 0, abort_flag, a.timeout_ns, false);
     }
+    // every MMA must be finished before TMEM is released
+    if (elect_one()) tc_commit(&bars->drain);
+    __syncwarp();
+    mbar_wait(&bars->drain, 0, abort_flag, a.timeout_ns, false);
   } else if (warp >= 4) {
     // ================= softmax: warps 4 + 4t .. 7 + 4t own tile t, one row per thread
     const int t = (warp - 4) >> 2;
     const int quad = warp & 3;       // TMEM lane quadrant this warp may access
     const int r = quad * 32 + lane;  // row within the tile
-    const TileJob job = t ? tj[1] : tj[0];  // selects, not a dynamic index (no local memory)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t s_addr = tmem + lane_off + (t ? C::COL_S1 : C::COL_S0);
     const uint32_t o_addr = tmem + lane_off + (t ? C::COL_O1 : C::COL_O0);
     const uint32_t p_tile = sP + t * C::P_BYTES;
-    const int q = job.q0 + r;
-    const int khi = row_key_limit(a, q);
-    const int klo = MASKS ? row_key_low(a, q) : 0;
-    float m = -INFINITY, l = 0.f;
+    int k = 0;         // this tile's visits over all units (barrier phases)
+    int nfin = 0;      // units in which this tile had visits (o_final phases)
     bool fail = false;  // a wait gave up (the warp decides as one)
-    int k = 0;          // this tile's visits so far
-    for (int kb = tile_next(t, 0); kb != kDone; kb = tile_next(t, kb + 1), ++k) {
-      if (__any_sync(0xffffffffu, !mbar_wait(&bars->s_full[t], k & 1, abort_flag, a.timeout_ns) || *abort_flag)) {
-        fail = true;
-        break;
-      }
-      tc_fence_after();
-      float s[BN];
-      const bool masked = block_needs_mask<BN, MASKS>(a, job, kb);
-      const float mx = load_scores<MASKS, BN>(s_addr, masked, khi - kb * BN, klo - kb * BN, a.scale_log2, s);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->s_free[t]);  // S_t may be overwritten
-      // exact running maximum: whenever it grows, O is rescaled before this block's P V,
-      // so the row's largest probability is exactly 1 and its bf16 rounding is exact
-      float alpha = 1.0f;
-      if (mx > m) {           // false while nothing is visible (mx = -inf)
-        alpha = ex2(m - mx);  // 0 when m = -inf
-        m = mx;
-      }
-      const float nmu = (m == -INFINITY) ? 0.0f : -m;
-      uint32_t P[BN / 2];
-      float a0 = 0.f, a1 = 0.f;
-      if (masked) {  // -inf entries: the exp unit returns exact zeros
-        exp_pairs<0u, BN / 2>(s, a.scale_log2, nmu, P, a0, a1);
-      } else {
-        exp_pairs<kEmuMask, BN / 2>(s, a.scale_log2, nmu, P, a0, a1);
-      }
-      l = l * alpha + (a0 + a1);
-      // P V of the previous visit must be done: it reads P_t, and O_t may be rescaled.
-      // (Warp-uniform decision: the stores and TMEM accesses below are per warp.)
-      if (!__all_sync(0xffffffffu, k == 0 || mbar_wait(&bars->o_done[t], (k - 1) & 1, abort_flag, a.timeout_ns))) {
-        fail = true;
-        break;
-      }
-      store_p_row<BN / 2>(p_tile, r, P);
-      fence_proxy_async_smem();
-      if (k > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+    for (int rd = 0; rd * (int)gridDim.x < a.n_units && !fail; ++rd) {
+      const int u = snake_unit(rd);
+      if (u >= a.n_units) continue;
+      unit_tiles<BN, MASKS>(a, u, b, kvh, tj);
+      const TileJob job = t ? tj[1] : tj[0];  // selects, not a dynamic index (no local memory)
+      const int q = job.q0 + r;
+      const int khi = row_key_limit(a, q);
+      const int klo = MASKS ? row_key_low(a, q) : 0;
+      float m = -INFINITY, l = 0.f;
+      int kl = 0;  // visits in this unit
+      for (int kb = tile_next(t, 0); kb != kDone; kb = tile_next(t, kb + 1), ++k, ++kl) {
+        if (__any_sync(0xffffffffu, !mbar_wait(&bars->s_full[t], k & 1, abort_flag, a.timeout_ns) || *abort_flag)) {
+          fail = true;
+          break;
+        }
         tc_fence_after();
-        rescale_cols<D>(o_addr, alpha);
-        tmem_st_wait();
+        float s[BN];
+        const bool masked = block_needs_mask<BN, MASKS>(a, job, kb);
+        const float mx = load_scores<MASKS, BN>(s_addr, masked, khi - kb * BN, klo - kb * BN, a.scale_log2, s);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free[t]);  // S_t may be overwritten
+        // exact running maximum: whenever it grows, O is rescaled before this block's P V,
+        // so the row's largest probability is exactly 1 and its bf16 rounding is exact
+        float alpha = 1.0f;
+        if (mx > m) {           // false while nothing is visible (mx = -inf)
+          alpha = ex2(m - mx);  // 0 when m = -inf
+          m = mx;
+        }
+        const float nmu = (m == -INFINITY) ? 0.0f : -m;
+        uint32_t P[BN / 2];
+        float a0 = 0.f, a1 = 0.f;
+        if (masked) {  // -inf entries: the exp unit returns exact zeros
+          exp_pairs<0u, BN / 2>(s, a.scale_log2, nmu, P, a0, a1);
+        } else {
+          exp_pairs<kEmuMask, BN / 2>(s, a.scale_log2, nmu, P, a0, a1);
+        }
+        l = l * alpha + (a0 + a1);
+        // P V of the tile's previous visit (of this unit or the last) must be done: it
+        // reads P_t, and O_t may be rescaled.  (Warp-uniform decision: the stores and
+        // TMEM accesses below are per warp.)
+        if (!__all_sync(0xffffffffu,
+                        k == 0 || mbar_wait(&bars->o_done[t], (k - 1) & 1, abort_flag, a.timeout_ns))) {
+          fail = true;
+          break;
+        }
+        store_p_row<BN / 2>(p_tile, r, P);
+        fence_proxy_async_smem();
+        if (kl > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+          tc_fence_after();
+          rescale_cols<D>(o_addr, alpha);
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[t]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[t]);
-    }
-    bool ok = !fail;
-    const bool have_o = k > 0;
-    if (ok && have_o) {
-      ok = mbar_wait(&bars->o_final[t], 0, abort_flag, a.timeout_ns);
-      tc_fence_after();
-    }
-    ok = __all_sync(0xffffffffu, ok);  // the TMEM loads of the epilogue are per warp
-    if (ok) {
+      if (fail) break;
+      const bool have_o = kl > 0;
+      bool ok = true;
+      if (have_o) {
+        // the unit's last P V; the next unit's first P V (which overwrites O_t) waits for
+        // this warp's next p_full, given after these TMEM loads
+        ok = mbar_wait(&bars->o_final[t], nfin & 1, abort_flag, a.timeout_ns);
+        tc_fence_after();
+        ++nfin;
+      }
+      ok = __all_sync(0xffffffffu, ok);  // the TMEM loads of the epilogue are per warp
+      if (!ok) {
+        fail = true;
+        break;
+      }
       const bool valid = r < job.rows;
       const size_t row = ((size_t)b * a.Hq + job.hq) * (size_t)a.Nq + (size_t)(valid ? q : 0);
       store_cols<D>(a, o_addr, have_o, valid, row * D, l);
