@@ -169,30 +169,6 @@ __device__ __forceinline__ void build_row_bitmap(const FwdArgs& a, const TileJob
   }
 }
 
-template <int D, int BN>
-__device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t sQ, uint32_t sK) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, BN, 0, 0);
-  const uint64_t da0 = smem_desc_sw128(sQ, 16, 1024);
-  const uint64_t db0 = smem_desc_sw128(sK, 16, 1024);
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint64_t da = da0 + (uint64_t)((((kk >> 2) * (128 * 128) + (kk & 3) * 32)) >> 4);
-    const uint64_t db = db0 + (uint64_t)((((kk >> 2) * (BN * 128) + (kk & 3) * 32)) >> 4);
-    mma_ss(s_tmem, da, db, idesc, kk > 0 ? 1u : 0u);
-  }
-}
-
-template <int D, int BN>
-__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t sV, bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
-  const uint64_t db0 = smem_desc_sw128(sV, BN * 128, 1024);
-#pragma unroll
-  for (int kk = 0; kk < BN / 16; ++kk) {
-    const uint64_t db = db0 + (uint64_t)((kk * (16 * 128)) >> 4);
-    mma_ts(o_tmem, p_tmem + kk * 8, db, idesc, (accumulate || kk > 0) ? 1u : 0u);
-  }
-}
-
 // Multiplies the calling thread's O row (D fp32 columns in TMEM) by alpha.
 template <int D>
 __device__ __forceinline__ void rescale_o(uint32_t o_taddr, float alpha) {
@@ -306,22 +282,9 @@ struct PingPongBars {
 };
 static_assert(sizeof(PingPongBars) <= PingPongCfg<128>::BAR_BYTES, "barrier area");
 
-// O_t += P_t V with P from shared memory: k-step kk covers keys 16kk..16kk+15 (64-key
-// chunk kk/4 of the K-major P tile, 32 bytes per step within it).
-template <int D, int BN>
-__device__ __forceinline__ void issue_pv_ss(uint32_t o_tmem, uint32_t sP, uint32_t sV, bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
-  const uint64_t da0 = smem_desc_sw128(sP, 16, 1024);
-  const uint64_t db0 = smem_desc_sw128(sV, BN * 128, 1024);
-#pragma unroll
-  for (int kk = 0; kk < BN / 16; ++kk) {
-    const uint64_t da = da0 + (uint64_t)((((kk >> 2) * (128 * 128)) + (kk & 3) * 32) >> 4);
-    const uint64_t db = db0 + (uint64_t)((kk * (16 * 128)) >> 4);
-    mma_ss(o_tmem, da, db, idesc, (accumulate || kk > 0) ? 1u : 0u);
-  }
-}
-
-// The same two products with descriptors as word pairs (the pair kernel's MMA warp).
+// S = Q K^T (SS, both K-major) and O += P V (SS, P K-major from shared memory, V
+// MN-major), descriptors as word pairs: k-step kk covers 16 elements of the contraction,
+// inside 64-element chunk kk/4 (32 bytes per step within a 128-byte swizzled row).
 template <int D, int BN>
 __device__ __forceinline__ void issue_qk_w(uint32_t s_tmem, Desc q, Desc k) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, BN, 0, 0);
@@ -338,6 +301,17 @@ __device__ __forceinline__ void issue_pv_w(uint32_t o_tmem, Desc p, Desc v, bool
   for (int kk = 0; kk < BN / 16; ++kk)
     mma_ss_w(o_tmem, p.lo + (uint32_t)((((kk >> 2) * (128 * 128)) + (kk & 3) * 32) >> 4), p.hi,
              v.lo + (uint32_t)((kk * (16 * 128)) >> 4), v.hi, idesc, (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// O += P V with P from TMEM (columns p_tmem + 8 kk for k-step kk), V descriptor as a
+// word pair (the d = 256 kernel).
+template <int D, int BN>
+__device__ __forceinline__ void issue_pv_ts_w(uint32_t o_tmem, uint32_t p_tmem, Desc v, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk)
+    mma_ts_w(o_tmem, p_tmem + kk * 8, v.lo + (uint32_t)((kk * (16 * 128)) >> 4), v.hi, idesc,
+             (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // A quarter of the probability pairs (kEmuMask) is computed on the FMA pipe (exp2_fma2)
@@ -1025,46 +999,66 @@ __global__ void __launch_bounds__(256, 1) attn_fwd_single_kernel(const __grid_co
     }
   } else if (warp == 1) {
     // Visit j: K at ring position 2j, V at 2j + 1; S(j) in TMEM block j & 1.  S(j + 2) is
-    // issued right after P V(j), which freed that block.
-    if (lane == 0 && any) {
+    // issued right after P V(j), which freed that block.  The whole warp runs the loop and
+    // one elected lane issues (see the two-tile kernel).
+    if (any) {
       auto stage_of = [&](int it) { return it % C::NSTAGE; };
       auto parity_of = [&](int it) { return (uint32_t)((it / C::NSTAGE) & 1); };
       auto colS = [&](int j) { return (j & 1) ? C::COL_S1 : C::COL_S0; };
-      bool ok = mbar_wait(&bars->q_full, 0, abort_flag, a.timeout_ns);
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.timeout_ns));
+      };
+      const Desc dq = desc_sw128(sQ, 16, 1024);
+      const Desc dk0 = desc_sw128(sKV, 16, 1024);
+      const Desc dv0 = desc_sw128(sKV, BN * 128, 1024);
+      auto kdesc = [&](int it) { return Desc{dk0.lo + (uint32_t)(stage_of(it) * (C::KV_BYTES >> 4)), dk0.hi}; };
+      auto vdesc = [&](int it) { return Desc{dv0.lo + (uint32_t)(stage_of(it) * (C::KV_BYTES >> 4)), dv0.hi}; };
+      bool ok = wait_all(&bars->q_full, 0);
       int nq = 0;      // Q K^T issued (visits 0 .. nq-1)
       int kbq = kb0;   // block of the next Q K^T
       for (; nq < 2 && kbq < job.jhi && ok; ++nq, kbq = next_visit<BN>(bits, job, kbq + 1)) {
         const int itK = 2 * nq;
-        if (!mbar_wait(&bars->kv_full[stage_of(itK)], parity_of(itK), abort_flag, a.timeout_ns)) {
+        if (!wait_all(&bars->kv_full[stage_of(itK)], parity_of(itK))) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        issue_qk<D, BN>(tmem + colS(nq), sQ, sKV + stage_of(itK) * C::KV_BYTES);
-        tc_commit(&bars->s_full[nq & 1]);
-        tc_commit(&bars->kv_empty[stage_of(itK)]);
+        if (elect_one()) {
+          tc_fence_after();
+          issue_qk_w<D, BN>(tmem + colS(nq), dq, kdesc(itK));
+          tc_commit(&bars->s_full[nq & 1]);
+          tc_commit(&bars->kv_empty[stage_of(itK)]);
+        }
+        __syncwarp();
       }
       for (int j = 0; j < nq && ok; ++j) {
         const int itV = 2 * j + 1;
-        if (!mbar_wait(&bars->kv_full[stage_of(itV)], parity_of(itV), abort_flag, a.timeout_ns)) break;
-        if (!mbar_wait(&bars->p_full[j & 1], (j >> 1) & 1, abort_flag, a.timeout_ns)) break;
-        tc_fence_after();
-        issue_pv<D, BN>(tmem + C::COL_O, tmem + colS(j), sKV + stage_of(itV) * C::KV_BYTES, j > 0);
-        tc_commit(&bars->o_done);
-        if (j + 1 == nq && kbq >= job.jhi) tc_commit(&bars->o_final);  // that was the last visit
-        tc_commit(&bars->kv_empty[stage_of(itV)]);
+        if (!wait_all(&bars->kv_full[stage_of(itV)], parity_of(itV))) break;
+        if (!wait_all(&bars->p_full[j & 1], (j >> 1) & 1)) break;
+        const bool last = j + 1 == nq && kbq >= job.jhi;  // that is the last visit
+        if (elect_one()) {
+          tc_fence_after();
+          issue_pv_ts_w<D, BN>(tmem + C::COL_O, tmem + colS(j), vdesc(itV), j > 0);
+          tc_commit(&bars->o_done);
+          if (last) tc_commit(&bars->o_final);
+          tc_commit(&bars->kv_empty[stage_of(itV)]);
+        }
+        __syncwarp();
         if (kbq < job.jhi) {
           const int itK = 2 * nq;  // nq == j + 2
-          if (!mbar_wait(&bars->kv_full[stage_of(itK)], parity_of(itK), abort_flag, a.timeout_ns)) break;
-          tc_fence_after();
-          issue_qk<D, BN>(tmem + colS(nq), sQ, sKV + stage_of(itK) * C::KV_BYTES);
-          tc_commit(&bars->s_full[nq & 1]);
-          tc_commit(&bars->kv_empty[stage_of(itK)]);
+          if (!wait_all(&bars->kv_full[stage_of(itK)], parity_of(itK))) break;
+          if (elect_one()) {
+            tc_fence_after();
+            issue_qk_w<D, BN>(tmem + colS(nq), dq, kdesc(itK));
+            tc_commit(&bars->s_full[nq & 1]);
+            tc_commit(&bars->kv_empty[stage_of(itK)]);
+          }
+          __syncwarp();
           ++nq;
           kbq = next_visit<BN>(bits, job, kbq + 1);
         }
       }
-      tc_commit(&bars->drain);
+      if (elect_one()) tc_commit(&bars->drain);
+      __syncwarp();
       mbar_wait(&bars->drain, 0, abort_flag, a.timeout_ns, false);
     }
   } else if (warp >= 4) {
