@@ -77,6 +77,15 @@ def csrc_digest() -> str:
     return h.hexdigest()[:16]
 
 
+# committed ncu summary of the prefill kernel, per workload
+PREFILL_PROFILES = {
+    "serving_step": "attn_fwd_pingpong_gqa_causal_2k.md",
+    "gqa_causal_2k": "attn_fwd_pingpong_gqa_causal_2k.md",
+    "gqa_causal_16k": "attn_fwd_pingpong_gqa_causal_16k.md",
+    "peaked_mha_d256": "attn_fwd_single_peaked_mha_d256.md",
+}
+
+
 def profiled_traffic(profile: str, scale: float = 1.0):
     """DRAM bytes per launch from a committed ncu summary, or None when the kernel sources
     changed since it was captured (its counters no longer describe this build)."""
@@ -412,8 +421,7 @@ def run_ours(args, dist):
     prefill_roofline = {
         "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
         "frac": achieved / peaks["bf16_tflops"],
-        "traffic": profiled_traffic("attn_fwd_pingpong_gqa_causal_2k.md")
-        if args.workload in ("serving_step", "gqa_causal_2k") else None,
+        "traffic": profiled_traffic(PREFILL_PROFILES[args.workload]) if args.workload in PREFILL_PROFILES else None,
         "peak_source": f"{peak_src} bf16_tflops (burst cuBLAS); frac of the sustained figure "
                        f"{achieved / peaks['bf16_tflops_sustained']:.3f}",
         "kernel": kname, "flops_per_launch": flops, "median_ms": statistics.median(pre_ms)}
