@@ -13,15 +13,17 @@
 // B200 design (not the pages' A100/H100 kernels):
 //   * Q, K and V tiles are brought in by TMA into 128-byte-swizzled shared memory and
 //     stream through a ring of stages guarded by mbarriers.
-//   * One thread issues tcgen05 MMAs: S = Q K^T lands in tensor memory (TMEM); the
-//     softmax warps read S from TMEM, write P (bf16) back over S, and the MMA
-//     O += P V takes P straight from TMEM; O accumulates in TMEM.
+//   * One warp issues the tcgen05 MMAs (one elected lane): S = Q K^T lands in tensor
+//     memory (TMEM), the softmax warps read S from TMEM, and O += P V accumulates in
+//     TMEM.
 //   * Kernel "pingpong" (d = 64 or 128): two 128-row Q tiles per CTA, each with its own
-//     softmax warpgroup, so one tile's softmax overlaps the other tile's MMAs (the
-//     FA4 page, section "Pipeline ping-pong avec double tuile Query", describes the same
-//     idea for Blackwell).  TMEM: S0 | S1 | O0 | O1 = 128 + 128 + d + d columns.
+//     softmax warpgroup (the FA4 page, section "Pipeline ping-pong avec double tuile
+//     Query", describes two Q tiles per CTA for Blackwell).  TMEM: S0 | S1 | O0 | O1 =
+//     128 + 128 + d + d columns.  P goes to shared memory, so S is free once the softmax
+//     has read it and the next S = Q K^T runs during the softmax.  Persistent CTAs.
 //   * Kernel "single" (d = 256): one Q tile, S double-buffered in TMEM (64 + 64 columns)
-//     next to O (256 columns), so the next S = Q K^T runs while the softmax works.
+//     next to O (256 columns), so the next S = Q K^T runs while the softmax works; P is
+//     written back over its S block and P V reads it from TMEM.
 //   * d <= 128: the reference of each row is its exact running maximum: whenever a block
 //     raises it, the row's O accumulator is rescaled in TMEM before the next P V.  The
 //     row's largest probability is then exactly 1 and its bf16 rounding is exact, which

@@ -68,12 +68,17 @@ CSRC = ("attn_api.cu", "decode_sm100.cuh", "prefill_sm100.cuh", "sm100_common.cu
 
 
 def csrc_digest() -> str:
-    """sha256 prefix of the kernel sources, to match against the committed ncu summaries."""
+    """sha256 prefix of the kernel sources without their comments and blank space, to match
+    against the committed ncu summaries (a comment edit does not change the kernels)."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for name in CSRC:
-        with open(os.path.join(ROOT, "attn_fwd_05_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "attn_fwd_05_b200", "csrc", name)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 
