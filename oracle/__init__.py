@@ -1,4 +1,4 @@
-"""fp64 CPU oracle for exact attention and paged-KV decode.
+"""fp64 CPU oracle for exact attention, its gradients and paged-KV decode.
 
 Test infrastructure: used only by the tests, the smoke check and the
 benchmark's CPU-baseline leg.  It shares no code with the CUDA library.
@@ -13,4 +13,6 @@ from .attention import (  # noqa: F401
     decode_paged,
     gather_pages,
     kv_head_of,
+    visible_mask,
 )
+from .backward import attention_backward, attention_head_backward  # noqa: F401
