@@ -8,6 +8,8 @@ library is loaded on first use and a missing or unloadable library raises
 
 from .binding import (  # noqa: F401
     AttnError,
+    attn_bwd,
+    attn_bwd_workspace_size,
     attn_decode_paged,
     attn_decode_paged_noalloc,
     attn_decode_paged_workspace_size,

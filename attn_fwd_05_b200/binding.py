@@ -32,6 +32,9 @@ SIGNATURES = {
     "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P]),
     "attn_fwd_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P]),
     "attn_fwd_masked": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _I, _P, _P]),
+    "attn_bwd_workspace_size": (ctypes.c_size_t, [_I, _I, _I]),
+    "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P,
+                      ctypes.c_size_t, _P]),
     "attn_decode_paged_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
     "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P,
                                ctypes.c_size_t, _P]),
@@ -152,6 +155,40 @@ def attn_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
     if o.dtype != torch.bfloat16:
         raise TypeError("attn_fwd writes bf16 o; use attn_fwd_ex for fp32")
     attn_fwd_ex(q, k, v, o, lse, causal, scale, stream)
+
+
+def attn_bwd_workspace_size(B: int, Hq: int, Nq: int) -> int:
+    return int(load_library().attn_bwd_workspace_size(B, Hq, Nq))
+
+
+def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, do: torch.Tensor,
+             lse: torch.Tensor, dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor, causal: bool, scale: float,
+             workspace: torch.Tensor | None = None, stream=None) -> None:
+    """Backward pass: fp32 dq [B, Hq, Nq, d], dk and dv [B, Hkv, Nk, d] from the bf16 inputs, the
+    forward's bf16 o and fp32 lse, and the bf16 upstream gradient do [B, Hq, Nq, d]."""
+    lib = load_library()
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if tuple(k.shape) != (B, Hkv, Nk, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k and v must be [B, Hkv, Nk, d] with q's B and d")
+    for name, t in (("o", o), ("do", do), ("dq", dq)):
+        if tuple(t.shape) != (B, Hq, Nq, d):
+            raise ValueError(f"{name} must be [B, Hq, Nq, d]")
+    for name, t in (("dk", dk), ("dv", dv)):
+        if tuple(t.shape) != (B, Hkv, Nk, d):
+            raise ValueError(f"{name} must be [B, Hkv, Nk, d]")
+    if tuple(lse.shape) != (B, Hq, Nq):
+        raise ValueError("lse must be [B, Hq, Nq]")
+    need = lib.attn_bwd_workspace_size(B, Hq, Nq)
+    if workspace is None:
+        workspace = torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
+    st = lib.attn_bwd(_dev(q, "q", torch.bfloat16, 4), _dev(k, "k", torch.bfloat16, 4), _dev(v, "v", torch.bfloat16, 4),
+                      _dev(o, "o", torch.bfloat16, 4), _dev(do, "do", torch.bfloat16, 4),
+                      _dev(lse, "lse", torch.float32, 3), _dev(dq, "dq", torch.float32, 4),
+                      _dev(dk, "dk", torch.float32, 4), _dev(dv, "dv", torch.float32, 4),
+                      B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
+                      _dev(workspace, "workspace", torch.uint8, 1), workspace.numel(), _stream(stream))
+    _check(st, "attn_bwd")
 
 
 def attn_decode_paged_workspace_size(num_seqs: int, Hq: int, Hkv: int, d: int, max_pages_per_seq: int,

@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "../../include/attn_b200.h"
+#include "backward_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "prefill_sm100.cuh"
 
@@ -122,6 +123,28 @@ attn_status launch_prefill(attn::FwdArgs& a, cudaStream_t st) {
   }
   return launch_status();
 }
+
+template <int D>
+attn_status launch_bwd(attn::BwdArgs& a, const void* o, const void* dout, float* delta, cudaStream_t st) {
+  using C = attn::BwdCfg<D>;
+  const long long rows = (long long)a.B * a.Hq * a.Nq;
+  const long long dblocks = std::min<long long>((rows + 7) / 8, (long long)sm_count() * 16);
+  attn::attn_bwd_delta_kernel<D><<<(unsigned)dblocks, 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), delta, rows);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  auto kkv = attn::attn_bwd_dkdv_kernel<D>;
+  auto kq = attn::attn_bwd_dq_kernel<D>;
+  const int slot = D == 64 ? 9 : 10;  // shared-memory slots 9-12: backward kernels
+  if (!ensure_smem(kkv, C::SMEM, slot) || !ensure_smem(kq, C::SMEM, slot + 2)) return ATTN_ERR_CUDA;
+  const long long gkv = (long long)a.B * a.Hkv * a.n_ktiles;
+  const long long gq = (long long)a.B * a.Hq * a.n_qtiles;
+  if (gkv > 0x7fffffffLL || gq > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  kkv<<<(unsigned)gkv, 256, C::SMEM, st>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  kq<<<(unsigned)gq, 256, C::SMEM, st>>>(a);
+  return launch_status();
+}
+
 
 template <int D>
 attn_status launch_decode(attn::DecArgs& a, cudaStream_t st, long long max_items) {
@@ -296,6 +319,70 @@ attn_status attn_fwd_masked(const void* q, const void* k, const void* v, void* o
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                      int Nq, int Nk, int d, float scale, int causal, void* stream) {
   return attn_fwd_ex(q, k, v, o, ATTN_DTYPE_BF16, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream);
+}
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Nq) {
+  if (B < 0 || Hq < 0 || Nq < 0) return 0;
+  return ((size_t)B * Hq * Nq * sizeof(float) + 255) & ~(size_t)255;
+}
+
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                     float* dq, float* dk, float* dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                     int causal, void* workspace, size_t workspace_bytes, void* stream) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0) return ATTN_OK;
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if ((long long)B * Hq > 0x7fffffffLL || (long long)B * Hkv > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (Nq == 0 && Nk == 0) return ATTN_OK;
+  if (Nq > 0 && (q == nullptr || o == nullptr || dout == nullptr || lse == nullptr || dq == nullptr))
+    return ATTN_ERR_INVALID_ARG;
+  if (Nk > 0 && (k == nullptr || v == nullptr || dk == nullptr || dv == nullptr)) return ATTN_ERR_INVALID_ARG;
+  if ((q && !aligned(q, 16)) || (k && !aligned(k, 16)) || (v && !aligned(v, 16)) || (o && !aligned(o, 16)) ||
+      (dout && !aligned(dout, 16)) || (lse && !aligned(lse, 4)) || (dq && !aligned(dq, 16)) ||
+      (dk && !aligned(dk, 16)) || (dv && !aligned(dv, 16)))
+    return ATTN_ERR_ALIGNMENT;
+  if (Nq == 0) {  // no query: no gradient reaches K or V
+    const size_t bytes = (size_t)B * Hkv * Nk * d * sizeof(float);
+    if (cudaMemsetAsync(dk, 0, bytes, st) != cudaSuccess || cudaMemsetAsync(dv, 0, bytes, st) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    return ATTN_OK;
+  }
+  if (Nk == 0) {  // no key: every output row is zero, so is its gradient
+    return cudaMemsetAsync(dq, 0, (size_t)B * Hq * Nq * d * sizeof(float), st) == cudaSuccess ? ATTN_OK
+                                                                                               : ATTN_ERR_CUDA;
+  }
+  const size_t need = attn_bwd_workspace_size(B, Hq, Nq);
+  if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return ATTN_ERR_ALIGNMENT;
+
+  attn::BwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  if (!encode_3d(&a.tm_q, q, d, Nq, (uint64_t)B * Hq, 128) || !encode_3d(&a.tm_do, dout, d, Nq, (uint64_t)B * Hq, 128) ||
+      !encode_3d(&a.tm_k, k, d, Nk, (uint64_t)B * Hkv, 128) || !encode_3d(&a.tm_v, v, d, Nk, (uint64_t)B * Hkv, 128))
+    return ATTN_ERR_CUDA;
+  a.lse = lse;
+  a.delta = static_cast<float*>(workspace);
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Nq = Nq;
+  a.Nk = Nk;
+  a.group = Hq / Hkv;
+  a.causal = causal;
+  a.n_qtiles = (Nq + 127) / 128;
+  a.n_ktiles = (Nk + 127) / 128;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.timeout_ns = kDefaultTimeoutNs;
+  float* delta = static_cast<float*>(workspace);
+  return d == 64 ? launch_bwd<64>(a, o, dout, delta, st) : launch_bwd<128>(a, o, dout, delta, st);
 }
 
 size_t attn_decode_paged_workspace_size(int num_seqs, int Hq, int Hkv, int d, int max_pages_per_seq,

@@ -284,38 +284,6 @@ struct PingPongBars {
 };
 static_assert(sizeof(PingPongBars) <= PingPongCfg<128>::BAR_BYTES, "barrier area");
 
-// S = Q K^T (SS, both K-major) and O += P V (SS, P K-major from shared memory, V
-// MN-major), descriptors as word pairs: k-step kk covers 16 elements of the contraction,
-// inside 64-element chunk kk/4 (32 bytes per step within a 128-byte swizzled row).
-template <int D, int BN>
-__device__ __forceinline__ void issue_qk_w(uint32_t s_tmem, Desc q, Desc k) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, BN, 0, 0);
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk)
-    mma_ss_w(s_tmem, q.lo + (uint32_t)((((kk >> 2) * (128 * 128)) + (kk & 3) * 32) >> 4), q.hi,
-             k.lo + (uint32_t)((((kk >> 2) * (BN * 128)) + (kk & 3) * 32) >> 4), k.hi, idesc, kk > 0 ? 1u : 0u);
-}
-
-template <int D, int BN>
-__device__ __forceinline__ void issue_pv_w(uint32_t o_tmem, Desc p, Desc v, bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
-#pragma unroll
-  for (int kk = 0; kk < BN / 16; ++kk)
-    mma_ss_w(o_tmem, p.lo + (uint32_t)((((kk >> 2) * (128 * 128)) + (kk & 3) * 32) >> 4), p.hi,
-             v.lo + (uint32_t)((kk * (16 * 128)) >> 4), v.hi, idesc, (accumulate || kk > 0) ? 1u : 0u);
-}
-
-// O += P V with P from TMEM (columns p_tmem + 8 kk for k-step kk), V descriptor as a
-// word pair (the d = 256 kernel).
-template <int D, int BN>
-__device__ __forceinline__ void issue_pv_ts_w(uint32_t o_tmem, uint32_t p_tmem, Desc v, bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
-#pragma unroll
-  for (int kk = 0; kk < BN / 16; ++kk)
-    mma_ts_w(o_tmem, p_tmem + kk * 8, v.lo + (uint32_t)((kk * (16 * 128)) >> 4), v.hi, idesc,
-             (accumulate || kk > 0) ? 1u : 0u);
-}
-
 // A quarter of the probability pairs (kEmuMask) is computed on the FMA pipe (exp2_fma2)
 // instead of the exp unit: per block the exp unit alone needs as many cycles as the
 // tensor core, the bottleneck the FA4 page names for Blackwell (section "Softmax

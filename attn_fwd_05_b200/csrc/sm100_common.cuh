@@ -231,6 +231,42 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Tile products with 128-byte swizzled operands written by TMA (64-element chunks of
+// 128-row tiles), descriptors as word pairs.  issue_qk_w: D(128 x BN) = A B^T, both
+// K-major, contraction D; issue_pv_w: D(128 x D) += A B, A K-major from shared memory,
+// B MN-major, contraction BN; issue_pv_ts_w: the same with A in TMEM.  k-step kk covers
+// 16 elements of the contraction, inside 64-element chunk kk/4 (32 bytes per step
+// within a 128-byte row) for a K-major operand, or 16 rows for an MN-major one.
+template <int D, int BN>
+__device__ __forceinline__ void issue_qk_w(uint32_t s_tmem, Desc q, Desc k) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, BN, 0, 0);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk)
+    mma_ss_w(s_tmem, q.lo + (uint32_t)((((kk >> 2) * (128 * 128)) + (kk & 3) * 32) >> 4), q.hi,
+             k.lo + (uint32_t)((((kk >> 2) * (BN * 128)) + (kk & 3) * 32) >> 4), k.hi, idesc, kk > 0 ? 1u : 0u);
+}
+
+template <int D, int BN>
+__device__ __forceinline__ void issue_pv_w(uint32_t o_tmem, Desc p, Desc v, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk)
+    mma_ss_w(o_tmem, p.lo + (uint32_t)((((kk >> 2) * (128 * 128)) + (kk & 3) * 32) >> 4), p.hi,
+             v.lo + (uint32_t)((kk * (16 * 128)) >> 4), v.hi, idesc, (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// O += P V with P from TMEM (columns p_tmem + 8 kk for k-step kk), V descriptor as a
+// word pair (the d = 256 kernel).
+template <int D, int BN>
+__device__ __forceinline__ void issue_pv_ts_w(uint32_t o_tmem, uint32_t p_tmem, Desc v, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk)
+    mma_ts_w(o_tmem, p_tmem + kk * 8, v.lo + (uint32_t)((kk * (16 * 128)) >> 4), v.hi, idesc,
+             (accumulate || kk > 0) ? 1u : 0u);
+}
+
+
 // Thread t of warp w reads lane 32*(w%4)+t, 32 consecutive 32-bit columns from taddr.
 #define ATTN_R32(r)                                                                                        \
   "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),           \

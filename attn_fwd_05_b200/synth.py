@@ -25,7 +25,7 @@ import torch
 _CHUNK = 1 << 24
 
 # stream ids: one independent generator per tensor
-_Q, _K, _V, _LENS, _PERM, _MASK = 1, 2, 3, 4, 5, 6
+_Q, _K, _V, _LENS, _PERM, _MASK, _DO = 1, 2, 3, 4, 5, 6, 7
 
 
 @dataclass(frozen=True)
@@ -167,6 +167,11 @@ def decode_inputs(shape: DecodeShape, seed: int, seq_lens: np.ndarray | None = N
     return PagedKV(q=q, k_pool=k_pool, v_pool=v_pool,
                    block_table=torch.from_numpy(table),
                    seq_lens=torch.from_numpy(seq_lens.copy()), page_size=s.page_size)
+
+
+def upstream_grad(shape: PrefillShape, seed: int) -> torch.Tensor:
+    """Seeded upstream gradient dO [B, Hq, Nq, d] for the backward pass: bf16 N(0, 1)."""
+    return normal_bf16((shape.B, shape.Hq, shape.Nq, shape.d), seed, _DO)
 
 
 def block_mask(Nq: int, Nk: int, density: float, seed: int, block: int = 128) -> torch.Tensor:

@@ -131,6 +131,40 @@ attn_status attn_fwd_masked(const void* q, const void* k, const void* v, void* o
                             void* stream);
 
 /*
+ * attn_bwd_workspace_size — bytes of scratch attn_bwd needs (one fp32 per query row for
+ * Delta = rowsum(dO o O)), rounded up to 256.  0 for negative sizes.
+ */
+size_t attn_bwd_workspace_size(int B, int Hq, int Nq);
+
+/*
+ * attn_bwd — gradients of attn_fwd with respect to Q, K and V (the backward pass).
+ *
+ * Source: patricehuetz.fr, "Flash Attention : pourquoi ton GPU utilise 85% de VRAM",
+ * section "Ce que fait Flash Attention" (second idea: the forward pass keeps no score
+ * matrix; the backward pass recomputes it block by block).  The gradients are those of
+ * O = softmax(scale Q K^T + mask) V for the upstream gradient dO, recomputed from Q, K
+ * and the forward's log-sum-exp:  dV = P^T dO, dS = P o (dO V^T - Delta),
+ * dQ = scale dS K, dK = scale dS^T Q, Delta_i = dO_i . O_i.
+ *
+ *   q, dout     device, bf16 [B, Hq, Nq, d]
+ *   k, v        device, bf16 [B, Hkv, Nk, d]
+ *   o, lse      device, the forward's outputs: bf16 O [B, Hq, Nq, d] and fp32 natural
+ *               log-sum-exp [B, Hq, Nq] (as written by attn_fwd on the same inputs)
+ *   dq          device, fp32 [B, Hq, Nq, d]   (written)
+ *   dk, dv      device, fp32 [B, Hkv, Nk, d]  (written; for grouped heads the sums over
+ *               the Hq/Hkv query heads that share the K/V head)
+ *   d           64 or 128 (256: ATTN_ERR_UNSUPPORTED);  causal as in attn_fwd.
+ *   workspace   device scratch of at least attn_bwd_workspace_size(B, Hq, Nq) bytes,
+ *               16-byte aligned, owned by the caller (ATTN_ERR_WORKSPACE if too small).
+ * Alignment: q, k, v, o, dout, dq, dk, dv 16-byte aligned.  A row with no visible key
+ * (lse = -inf) gets zero gradient.  Nq = 0 writes dk = dv = 0; Nk = 0 writes dq = 0.
+ */
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, float* dq, float* dk, float* dv, int B, int Hq, int Hkv,
+                     int Nq, int Nk, int d, float scale, int causal, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/*
  * attn_decode_paged_workspace_size — bytes of scratch attn_decode_paged needs for
  * these sizes (fp32 partial outputs and partial log-sum-exps of the split-K pass).
  * Returns 0 for sizes attn_decode_paged would reject.
