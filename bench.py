@@ -55,7 +55,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="serving_step",
-                   choices=["serving_step", "gqa_causal_16k", "peaked_mha_d256", "tiny_mha_d64", "gqa_causal_2k"])
+                   choices=["serving_step", "gqa_causal_16k", "peaked_mha_d256", "tiny_mha_d64", "gqa_causal_2k",
+                            "gqa_causal_2k_bwd", "gqa_causal_16k_bwd"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="bounded CPU-baseline sample length")
@@ -349,6 +350,115 @@ def config_block(args, shape):
     return cfg
 
 
+def run_backward(args, dist):
+    """Backward pass (attn_bwd: delta, dK/dV and dQ kernels) on a prefill workload.  FLOPs are
+    the method's five products, 2.5x the forward's (causal halved), as the pages' FA figures
+    count them; the dQ kernel's recomputation of S and dP is not counted."""
+    import attn_fwd_05_b200 as ab
+    ab.load_library()
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    name = args.workload[: -len("_bwd")]
+    shape = synth.WORKLOADS[name]
+    seed = rank_seed(synth.workload_seed(name), dist.rank)
+    pre = make_prefill(shape, seed, dev)
+    qd, kd, vd = pre["dev"]
+    do = synth.upstream_grad(shape, seed).to(dev)
+    scale = synth.default_scale(shape.d)
+    stream = torch.cuda.current_stream(dev)
+    ab.attn_fwd(qd, kd, vd, pre["o"], pre["lse"], shape.causal, scale, stream)
+    dq = torch.empty((shape.B, shape.Hq, shape.Nq, shape.d), dtype=torch.float32, device=dev)
+    dk = torch.empty((shape.B, shape.Hkv, shape.Nk, shape.d), dtype=torch.float32, device=dev)
+    dv = torch.empty_like(dk)
+    ws = torch.empty(ab.attn_bwd_workspace_size(shape.B, shape.Hq, shape.Nq), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flops = 2.5 * counts.prefill_flops(shape.B, shape.Hq, shape.Nq, shape.Nk, shape.d, shape.causal)
+
+    def step():
+        ab.attn_bwd(qd, kd, vd, pre["o"], do, pre["lse"], dq, dk, dv, shape.causal, scale, ws, stream)
+
+    clocks = ClockSampler(dist.local)
+    clocks.start()
+    for _ in range(args.warmup):
+        step()
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K)]
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        flush.zero_()
+        ev[2 * i].record(stream)
+        step()
+        ev[2 * i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clk = clocks.stop()
+    st = ab.attn_get_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"kernel fault in the timed region: {ab.attn_status_string(st)}")
+    ms = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K)]
+    tot = dist.max(sum(ms))
+    achieved = flops / (sum(ms) / K * 1e-3) / 1e12
+    line = {
+        "metric": "attn bwd TFLOPS & % of BF16 tensor peak", "value": dist.world * flops * K / (tot * 1e-3) / 1e12,
+        "unit": "TFLOP/s", "n_gpus": dist.world, "steps": K, "warmup": args.warmup, "ms_per_step": tot / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload,
+                   "prefill": {"B": shape.B, "Hq": shape.Hq, "Hkv": shape.Hkv, "Nq": shape.Nq, "Nk": shape.Nk,
+                               "d": shape.d, "causal": shape.causal},
+                   "l2": "L2 flushed between steps by writing a 256 MB buffer",
+                   "parallelism": f"independent replicas x{dist.world} (no data-path collective)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops (burst cuBLAS)",
+                     "kernel": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel + attn_bwd_delta_kernel (one call)",
+                     "flops_per_launch": flops, "median_ms": statistics.median(ms)},
+        "gpu_launches": 3 * K, "clocks": clk,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_backward_sample(shape, pre["host"], do.cpu(), scale, flops, args.cpu_seconds)
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def oracle_backward_sample(shape, host, do, scale, flops, seconds):
+    """The fp64 backward oracle on whole (batch, query head) pairs until about `seconds`
+    have passed, scaled to the workload's FLOPs by the share of heads done."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_limits
+        limit = threadpool_limits(1)  # the matrix products of numpy's BLAS on one thread
+    except Exception:
+        limit = None
+    q, k, v = host
+    G = shape.Hq // shape.Hkv
+    t0 = time.perf_counter()
+    heads = 0
+    done = False
+    for b in range(shape.B):
+        for h in range(shape.Hq):
+            kv = h // G
+            oracle.attention_head_backward(oracle.as_f64(q[b, h]), oracle.as_f64(k[b, kv]), oracle.as_f64(v[b, kv]),
+                                           oracle.as_f64(do[b, h]), scale, shape.causal)
+            heads += 1
+            if time.perf_counter() - t0 > seconds:
+                done = True
+                break
+        if done:
+            break
+    dt = time.perf_counter() - t0
+    if limit is not None:
+        limit.unregister()
+    share = heads / (shape.B * shape.Hq)
+    return {"value": flops * share / dt / 1e12, "unit": "TFLOP/s", "cores": 1 if limit is not None else os.cpu_count(),
+            "kind": "oracle",
+            "sample": f"{heads} of {shape.B * shape.Hq} (batch, head) pairs, fp64 backward, one thread, {dt:.1f} s"}
+
+
 def run_ours(args, dist):
     import attn_fwd_05_b200 as ab
     ab.load_library()
@@ -525,6 +635,8 @@ def main():
         return run_reference(args, dist)
     dist.init("nccl")
     try:
+        if args.workload.endswith("_bwd"):
+            return run_backward(args, dist)
         return run_ours(args, dist)
     finally:
         dist.close()

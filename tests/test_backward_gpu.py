@@ -135,3 +135,35 @@ def test_backward_rejects_d256(cuda_device):
     g = torch.zeros((1, 1, 16, 256), device=dev)
     with pytest.raises(ab.AttnError):
         ab.attn_bwd(x, x, x, x, x, torch.zeros((1, 1, 16), device=dev), g, g, g, False, 0.1)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["gqa_causal_2k"])
+def test_backward_full_size_one_group(name, cuda_device):
+    # the whole workload on the GPU; the oracle on the query heads of one K/V head
+    s = synth.WORKLOADS[name]
+    seed = synth.workload_seed(name)
+    q, k, v = synth.prefill_inputs(s, seed)
+    do = synth.upstream_grad(s, seed)
+    scale = synth.default_scale(s.d)
+    dev = torch.device("cuda:0")
+    qd, kd, vd, dod = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
+    o = torch.empty((s.B, s.Hq, s.Nq, s.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((s.B, s.Hq, s.Nq), dtype=torch.float32, device=dev)
+    ab.attn_fwd(qd, kd, vd, o, lse, s.causal, scale)
+    dq = torch.empty((s.B, s.Hq, s.Nq, s.d), dtype=torch.float32, device=dev)
+    dk = torch.empty((s.B, s.Hkv, s.Nk, s.d), dtype=torch.float32, device=dev)
+    dv = torch.empty_like(dk)
+    ab.attn_bwd(qd, kd, vd, o, dod, lse, dq, dk, dv, s.causal, scale)
+    assert ab.attn_get_device_status() == 0
+    b, kv = s.B - 1, s.Hkv - 1
+    G = s.Hq // s.Hkv
+    heads = list(range(kv * G, (kv + 1) * G))
+    sub = lambda t, hs: t[b:b + 1, hs]  # noqa: E731
+    ref, bnd = reference_and_bounds(sub(q, heads), sub(k, [kv]), sub(v, [kv]), sub(do, heads), scale, s.causal,
+                                    o[b:b + 1, heads].double().cpu().numpy())
+    got = (dq[b:b + 1, heads].double().cpu().numpy(), dk[b:b + 1, [kv]].double().cpu().numpy(),
+           dv[b:b + 1, [kv]].double().cpu().numpy())
+    for name_, g, r, e in zip(("dq", "dk", "dv"), got, ref, bnd):
+        err = np.abs(g - r)
+        assert not (err > e + 1e-6 * np.abs(r).max()).any(), f"{name_}: max excess {(err - e).max():.3e}"
