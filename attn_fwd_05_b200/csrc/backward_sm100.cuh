@@ -184,8 +184,10 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dkdv_kernel(const __grid_cons
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int kt = blockIdx.x % a.n_ktiles;
-  const int bkv = blockIdx.x / a.n_ktiles;  // b * Hkv + kvh
+  // causal: the first K/V tiles are seen by the most q-tiles, so they go first (longest
+  // processing time first); consecutive CTAs share a key-tile index
+  const int kt = blockIdx.x / (a.B * a.Hkv);
+  const int bkv = blockIdx.x % (a.B * a.Hkv);  // b * Hkv + kvh
   const int b = bkv / a.Hkv, kvh = bkv % a.Hkv;
   const int k0 = kt * 128;
   const int qt_lo = kv_qt_lo(a, kt);
@@ -365,8 +367,9 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dq_kernel(const __grid_consta
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int qt = blockIdx.x % a.n_qtiles;
-  const int bh = blockIdx.x / a.n_qtiles;  // b * Hq + hq
+  // causal: the last q-tiles see the most K/V tiles, so they go first
+  const int qt = a.n_qtiles - 1 - (int)(blockIdx.x / (a.B * a.Hq));
+  const int bh = blockIdx.x % (a.B * a.Hq);  // b * Hq + hq
   const int b = bh / a.Hq, hq = bh % a.Hq;
   const int bkv = b * a.Hkv + hq / a.group;
   const int q0 = qt * 128;
