@@ -16,3 +16,4 @@ from .attention import (  # noqa: F401
     visible_mask,
 )
 from .backward import attention_backward, attention_head_backward  # noqa: F401
+from .fp8 import attention_fp8_reference, block_quantize, dequantize, e4m3_value, quantize_e4m3  # noqa: F401
