@@ -15,8 +15,10 @@ from .binding import (  # noqa: F401
     attn_decode_paged_workspace_size,
     attn_fwd,
     attn_fwd_ex,
+    attn_fwd_fp8,
     attn_fwd_masked,
     attn_get_device_status,
+    attn_quantize_fp8,
     attn_debug_exp2,
     attn_debug_watchdog,
     attn_status_string,

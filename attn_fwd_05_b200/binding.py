@@ -32,6 +32,8 @@ SIGNATURES = {
     "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P]),
     "attn_fwd_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P]),
     "attn_fwd_masked": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _I, _P, _P]),
+    "attn_quantize_fp8": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
+    "attn_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P]),
     "attn_bwd_workspace_size": (ctypes.c_size_t, [_I, _I, _I]),
     "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P,
                       ctypes.c_size_t, _P]),
@@ -155,6 +157,47 @@ def attn_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
     if o.dtype != torch.bfloat16:
         raise TypeError("attn_fwd writes bf16 o; use attn_fwd_ex for fp32")
     attn_fwd_ex(q, k, v, o, lse, causal, scale, stream)
+
+
+def attn_quantize_fp8(x: torch.Tensor, block_rows: int, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Block e4m3 quantization of a bf16 [..., N, d] tensor: returns (codes uint8 [..., N, d],
+    scales fp32 [..., ceil(N / block_rows)])."""
+    lib = load_library()
+    *lead, N, d = x.shape
+    planes = 1
+    for n in lead:
+        planes *= n
+    nblk = (N + block_rows - 1) // block_rows
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scales = torch.empty((*lead, nblk), dtype=torch.float32, device=x.device)
+    st = lib.attn_quantize_fp8(_dev(x, "x", torch.bfloat16), out.data_ptr(), scales.data_ptr(), planes, N, d,
+                               block_rows, _stream(stream))
+    _check(st, "attn_quantize_fp8")
+    return out, scales
+
+
+def attn_fwd_fp8(q8, q_scale, k8, k_scale, v8, v_scale, o, lse, causal: bool, scale: float, stream=None) -> None:
+    """FP8 forward: e4m3 q8 [B, Hq, Nq, 128], k8/v8 [B, Hkv, Nk, 128] (uint8 tensors) with fp32
+    scales q_scale [B, Hq, ceil(Nq/128)], k_scale [B, Hkv, ceil(Nk/128)], v_scale [B, Hkv]."""
+    lib = load_library()
+    B, Hq, Nq, d = q8.shape
+    Hkv, Nk = k8.shape[1], k8.shape[2]
+    if tuple(k8.shape) != (B, Hkv, Nk, d) or tuple(v8.shape) != tuple(k8.shape):
+        raise ValueError("k8 and v8 must be [B, Hkv, Nk, d]")
+    if tuple(q_scale.shape) != (B, Hq, (Nq + 127) // 128) or tuple(k_scale.shape) != (B, Hkv, (Nk + 127) // 128) \
+            or tuple(v_scale.shape) != (B, Hkv):
+        raise ValueError("scale shapes must be [B, Hq, ceil(Nq/128)], [B, Hkv, ceil(Nk/128)], [B, Hkv]")
+    if tuple(o.shape) != (B, Hq, Nq, d):
+        raise ValueError("o must be [B, Hq, Nq, d]")
+    odt = DTYPE_BF16 if o.dtype == torch.bfloat16 else DTYPE_F32 if o.dtype == torch.float32 else None
+    if odt is None:
+        raise TypeError("o must be bf16 or fp32")
+    st = lib.attn_fwd_fp8(_dev(q8, "q8", torch.uint8, 4), _dev(q_scale, "q_scale", torch.float32, 3),
+                          _dev(k8, "k8", torch.uint8, 4), _dev(k_scale, "k_scale", torch.float32, 3),
+                          _dev(v8, "v8", torch.uint8, 4), _dev(v_scale, "v_scale", torch.float32, 2),
+                          _dev(o, "o", o.dtype, 4), odt, None if lse is None else _dev(lse, "lse", torch.float32, 3),
+                          B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), _stream(stream))
+    _check(st, "attn_fwd_fp8")
 
 
 def attn_bwd_workspace_size(B: int, Hq: int, Nq: int) -> int:

@@ -17,6 +17,7 @@
 #include "backward_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "prefill_sm100.cuh"
+#include "fwd_fp8_sm100.cuh"
 
 namespace {
 
@@ -51,6 +52,20 @@ bool encode_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows
   cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// e4m3 tensors [outer, rows, 128 bytes]: one 128-byte swizzled row per token.
+bool encode_3d_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {128, rows, outer};
+  cuuint64_t strides[2] = {128, rows * 128};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -319,6 +334,77 @@ attn_status attn_fwd_masked(const void* q, const void* k, const void* v, void* o
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                      int Nq, int Nk, int d, float scale, int causal, void* stream) {
   return attn_fwd_ex(q, k, v, o, ATTN_DTYPE_BF16, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream);
+}
+
+attn_status attn_quantize_fp8(const void* x, void* out, float* scales, int planes, int N, int d, int block_rows,
+                              void* stream) {
+  if (planes < 0 || N < 0 || d <= 0 || (d & 1) || block_rows <= 0) return ATTN_ERR_INVALID_ARG;
+  if (planes == 0 || N == 0) return ATTN_OK;
+  if (x == nullptr || out == nullptr || scales == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(x, 4) || !aligned(out, 2) || !aligned(scales, 4)) return ATTN_ERR_ALIGNMENT;
+  const long long nblk = ((long long)N + block_rows - 1) / block_rows;
+  const long long grid = (long long)planes * nblk;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  attn::attn_quantize_e4m3_kernel<<<(unsigned)grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<uint8_t*>(out), scales, N, d, block_rows, (int)nblk);
+  return launch_status();
+}
+
+attn_status attn_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const float* k_scale, const void* v8,
+                         const float* v_scale, void* o, int o_dtype, float* lse, int B, int Hq, int Hkv, int Nq, int Nk,
+                         int d, float scale, int causal, void* stream) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (o_dtype != ATTN_DTYPE_BF16 && o_dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || Nq == 0) return ATTN_OK;
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (q8 == nullptr || q_scale == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (Nk > 0 && (k8 == nullptr || v8 == nullptr || k_scale == nullptr || v_scale == nullptr))
+    return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q8, 16) || !aligned(o, 16) || (Nk > 0 && (!aligned(k8, 16) || !aligned(v8, 16))) ||
+      (lse != nullptr && !aligned(lse, 4)))
+    return ATTN_ERR_ALIGNMENT;
+  if ((long long)B * Hq > 0x7fffffffLL || (long long)B * Hkv > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int o_f32 = o_dtype == ATTN_DTYPE_F32;
+  if (Nk == 0) {
+    attn::attn_fwd_empty_kernel<<<592, 256, 0, st>>>(o, lse, (size_t)B * Hq * Nq, d, o_f32);
+    return launch_status();
+  }
+  attn::Fp8Args a;
+  std::memset(&a, 0, sizeof(a));
+  if (!encode_3d_u8(&a.tm_q, q8, Nq, (uint64_t)B * Hq) || !encode_3d_u8(&a.tm_k, k8, Nk, (uint64_t)B * Hkv) ||
+      !encode_3d_u8(&a.tm_v, v8, Nk, (uint64_t)B * Hkv))
+    return ATTN_ERR_CUDA;
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Nq = Nq;
+  a.Nk = Nk;
+  a.group = Hq / Hkv;
+  a.causal = causal;
+  a.o_f32 = o_f32;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.pair_heads = (a.group % 2 == 0) ? 1 : 0;
+  a.n_qtiles = (Nq + 127) / 128;
+  a.n_ktiles = (Nk + 127) / 128;
+  a.timeout_ns = kDefaultTimeoutNs;
+  const long long qp = (a.n_qtiles + 1) / 2;
+  const long long units = a.pair_heads ? (long long)B * (Hq / 2) * a.n_qtiles : (long long)B * Hq * qp;
+  if (units <= 0 || units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  a.n_units = (int)units;
+  using C = attn::Fp8Cfg;
+  if (!ensure_smem(attn::attn_fwd_fp8_kernel, C::SMEM, 13)) return ATTN_ERR_CUDA;
+  const long long grid = std::min<long long>(units, sm_count());
+  attn::attn_fwd_fp8_kernel<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(a);
+  return launch_status();
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int Nq) {

@@ -56,7 +56,7 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="serving_step",
                    choices=["serving_step", "gqa_causal_16k", "peaked_mha_d256", "tiny_mha_d64", "gqa_causal_2k",
-                            "gqa_causal_2k_bwd", "gqa_causal_16k_bwd"])
+                            "gqa_causal_2k_bwd", "gqa_causal_16k_bwd", "gqa_causal_2k_fp8", "gqa_causal_16k_fp8"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="bounded CPU-baseline sample length")
@@ -459,6 +459,78 @@ def oracle_backward_sample(shape, host, do, scale, flops, seconds):
             "sample": f"{heads} of {shape.B * shape.Hq} (batch, head) pairs, fp64 backward, one thread, {dt:.1f} s"}
 
 
+def run_fp8(args, dist):
+    """FP8 forward (attn_fwd_fp8) on a d = 128 prefill workload: inputs quantized on the GPU
+    once (Q, K per 128 rows, V per head), outside the timed region.  The tensor peak for
+    e4m3 is the measured bf16 figure times the nominal dense ratio 4.5 / 2.25 = 2."""
+    import attn_fwd_05_b200 as ab
+    ab.load_library()
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    name = args.workload[: -len("_fp8")]
+    shape = synth.WORKLOADS[name]
+    seed = rank_seed(synth.workload_seed(name), dist.rank)
+    pre = make_prefill(shape, seed, dev)
+    qd, kd, vd = pre["dev"]
+    q8, qs = ab.attn_quantize_fp8(qd, 128)
+    k8, ks = ab.attn_quantize_fp8(kd, 128)
+    v8, vs = ab.attn_quantize_fp8(vd, shape.Nk)
+    vs = vs[..., 0].contiguous()
+    scale = synth.default_scale(shape.d)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flops = counts.prefill_flops(shape.B, shape.Hq, shape.Nq, shape.Nk, shape.d, shape.causal)
+
+    def step():
+        ab.attn_fwd_fp8(q8, qs, k8, ks, v8, vs, pre["o"], pre["lse"], shape.causal, scale, stream)
+
+    clocks = ClockSampler(dist.local)
+    clocks.start()
+    for _ in range(args.warmup):
+        step()
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K)]
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        flush.zero_()
+        ev[2 * i].record(stream)
+        step()
+        ev[2 * i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clk = clocks.stop()
+    st = ab.attn_get_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"kernel fault in the timed region: {ab.attn_status_string(st)}")
+    ms = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K)]
+    tot = dist.max(sum(ms))
+    achieved = flops / (sum(ms) / K * 1e-3) / 1e12
+    peak = 2.0 * peaks["bf16_tflops"]
+    line = {
+        "metric": "attn fwd TFLOPS (e4m3 inputs) & % of FP8 tensor peak",
+        "value": dist.world * flops * K / (tot * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": dist.world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": tot / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": args.workload,
+                   "prefill": {"B": shape.B, "Hq": shape.Hq, "Hkv": shape.Hkv, "Nq": shape.Nq, "Nk": shape.Nk,
+                               "d": shape.d, "causal": shape.causal},
+                   "l2": "L2 flushed between steps by writing a 256 MB buffer",
+                   "parallelism": f"independent replicas x{dist.world} (no data-path collective)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"2 x {peak_src} bf16_tflops (nominal e4m3 : bf16 dense ratio)",
+                     "kernel": "attn_fwd_fp8_kernel", "flops_per_launch": flops, "median_ms": statistics.median(ms)},
+        "gpu_launches": K, "clocks": clk,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_ours(args, dist):
     import attn_fwd_05_b200 as ab
     ab.load_library()
@@ -637,6 +709,8 @@ def main():
     try:
         if args.workload.endswith("_bwd"):
             return run_backward(args, dist)
+        if args.workload.endswith("_fp8"):
+            return run_fp8(args, dist)
         return run_ours(args, dist)
     finally:
         dist.close()

@@ -131,6 +131,42 @@ attn_status attn_fwd_masked(const void* q, const void* k, const void* v, void* o
                             void* stream);
 
 /*
+ * attn_quantize_fp8 — block quantization of a bf16 tensor to e4m3 (FP8), for attn_fwd_fp8.
+ *
+ * Source: polydesk.ai glossary "FlashAttention", section on FlashAttention-3 (FP8 inputs
+ * with one scale per block).  Format: e4m3 of the OCP 8-bit floating-point format
+ * (largest finite value 448).  For each block of `block_rows` consecutive rows of a
+ * plane: scale = amax / 448 (1 for an all-zero block), code = x / scale rounded to the
+ * nearest e4m3 value (ties to even, saturating at 448, the sign kept when a value rounds
+ * to zero); both divisions are fp32 with round-to-nearest.
+ *
+ *   x        device, bf16 [planes, N, d] (d even), read-only, 4-byte aligned
+ *   out      device, e4m3 bytes [planes, N, d] (written), 2-byte aligned
+ *   scales   device, fp32 [planes, ceil(N / block_rows)] (written)
+ * attn_fwd_fp8 takes Q and K with block_rows = 128 and V with block_rows = N.
+ */
+attn_status attn_quantize_fp8(const void* x, void* out, float* scales, int planes, int N, int d,
+                              int block_rows, void* stream);
+
+/*
+ * attn_fwd_fp8 — attn_fwd_ex with FP8 (e4m3) Q, K and V and block scales (d = 128).
+ *
+ * Computes the attention of the dequantized inputs (code x scale of its block):
+ *   q8, k8, v8  device, e4m3 [B, Hq, Nq, 128] / [B, Hkv, Nk, 128], 16-byte aligned
+ *   q_scale     device, fp32 [B, Hq, ceil(Nq/128)]: one scale per 128 query rows
+ *   k_scale     device, fp32 [B, Hkv, ceil(Nk/128)]: one scale per 128 keys
+ *   v_scale     device, fp32 [B, Hkv]: one scale per head
+ *   o, lse, causal, scale and the other sizes as in attn_fwd_ex.
+ * The probabilities are rounded to e4m3 (after a factor 256, exact in the format, so a
+ * row's largest probability is exact) before P V; the log-sum-exp uses their fp32 sum.
+ * d other than 128: ATTN_ERR_UNSUPPORTED.
+ */
+attn_status attn_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const float* k_scale,
+                         const void* v8, const float* v_scale, void* o, int o_dtype, float* lse,
+                         int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                         void* stream);
+
+/*
  * attn_bwd_workspace_size — bytes of scratch attn_bwd needs (one fp32 per query row for
  * Delta = rowsum(dO o O)), rounded up to 256.  0 for negative sizes.
  */
