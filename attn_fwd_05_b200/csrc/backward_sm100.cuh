@@ -127,8 +127,8 @@ struct BwdBars {
   uint64_t fixed_full;  // the CTA's own tiles (K and V, or Q and dO) have landed
   uint64_t stage_full[2];
   uint64_t stage_empty[2];
-  uint64_t s_full;      // the two score-like products of the step are in TMEM
-  uint64_t p_full;      // P and/or dS written back (4 warps)
+  uint64_t s_full[2];   // half h of the step's two score-like products is in TMEM
+  uint64_t p_full[2];   // P and/or dS of half h written back (4 warps)
   uint64_t o_final;     // the last accumulation is done
   uint64_t drain;
   uint32_t tmem_base;
@@ -145,7 +145,9 @@ struct BwdCfg {
   static constexpr int OFF_BAR = OFF_STAT + 2 * 2 * 128 * 4;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + 1 KB alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
+  // S and dP in two 64-column halves each (half h at +64h), then the accumulators
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC0 = 256, COL_ACC1 = 256 + D;
+  static constexpr int HALF_ROWS_BYTES = 64 * 128;  // offset of rows 64.. inside a 64-column chunk
 };
 
 __device__ __forceinline__ void bwd_init_bars(BwdBars* bars, int stage_full_count) {
@@ -154,8 +156,10 @@ __device__ __forceinline__ void bwd_init_bars(BwdBars* bars, int stage_full_coun
     mbar_init(&bars->stage_full[s], stage_full_count);
     mbar_init(&bars->stage_empty[s], 1);
   }
-  mbar_init(&bars->s_full, 1);
-  mbar_init(&bars->p_full, 4);
+  for (int h = 0; h < 2; ++h) {
+    mbar_init(&bars->s_full[h], 1);
+    mbar_init(&bars->p_full[h], 4);
+  }
   mbar_init(&bars->o_final, 1);
   mbar_init(&bars->drain, 1);
   bars->abort_flag = 0;
@@ -268,30 +272,54 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dkdv_kernel(const __grid_cons
     };
     if (nsteps > 0) {
       const Desc dk = desc_sw128(sK, 16, 1024), dvk = desc_sw128(sV, 16, 1024);
-      bool ok = wait_all(&bars->fixed_full, 0);
+      // Each step is split in two halves of 64 queries, so that the softmax warps work on
+      // one half while the tensor core computes the other:
+      //   S^T_h = K Q_h^T, dP^T_h = V dO_h^T  (64 columns each), then after p_full[h]
+      //   dV += P^T_h dO_h, dK += dS^T_h Q_h  (contraction over the half's 64 queries).
+      // The next step's half h overwrites P_h / dS_h only after those products were
+      // issued (this thread issues in order).
+      auto stage_q = [&](int j) { return sRing + (j & 1) * 2 * C::TILE_BYTES; };
+      auto issue_s = [&](int j, int h) {
+        const uint32_t sQ = stage_q(j) + h * C::HALF_ROWS_BYTES, sDO = sQ + C::TILE_BYTES;
+        if (elect_one()) {
+          tc_fence_after();
+          issue_qk_rows<D, 64>(tmem + C::COL_S + 64 * h, dk, desc_sw128(sQ, 16, 1024));
+          issue_qk_rows<D, 64>(tmem + C::COL_DP + 64 * h, dvk, desc_sw128(sDO, 16, 1024));
+          tc_commit(&bars->s_full[h]);
+        }
+        __syncwarp();
+      };
+      auto issue_acc = [&](int j, int h) {
+        const uint32_t sQ = stage_q(j) + h * C::HALF_ROWS_BYTES, sDO = sQ + C::TILE_BYTES;
+        const bool acc = j > 0 || h > 0;
+        if (elect_one()) {
+          tc_fence_after();
+          issue_pv_ts_w<D, 64>(tmem + C::COL_ACC1, tmem + C::COL_S + 64 * h, desc_sw128(sDO, 128 * 128, 1024), acc);
+          issue_pv_ts_w<D, 64>(tmem + C::COL_ACC0, tmem + C::COL_DP + 64 * h, desc_sw128(sQ, 128 * 128, 1024), acc);
+        }
+        __syncwarp();
+      };
+      bool ok = wait_all(&bars->fixed_full, 0) && wait_all(&bars->stage_full[0], 0);
+      if (ok) {
+        issue_s(0, 0);
+        issue_s(0, 1);
+      }
       for (int j = 0; j < nsteps && ok; ++j) {
-        const int st = j & 1;
-        const uint32_t sQ = sRing + st * 2 * C::TILE_BYTES, sDO = sQ + C::TILE_BYTES;
-        if (!wait_all(&bars->stage_full[st], (j >> 1) & 1)) break;
-        // S^T = K Q^T and dP^T = V dO^T (the softmax warps have read the previous step's
-        // values before the previous p_full, and this thread issues in order)
+        const bool more = j + 1 < nsteps;
+        if (!wait_all(&bars->p_full[0], j & 1)) break;
+        issue_acc(j, 0);
+        if (more) {
+          if (!wait_all(&bars->stage_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) break;
+          issue_s(j + 1, 0);
+        }
+        if (!wait_all(&bars->p_full[1], j & 1)) break;
+        issue_acc(j, 1);
         if (elect_one()) {
-          tc_fence_after();
-          issue_qk_w<D, 128>(tmem + C::COL_S, dk, desc_sw128(sQ, 16, 1024));
-          issue_qk_w<D, 128>(tmem + C::COL_DP, dvk, desc_sw128(sDO, 16, 1024));
-          tc_commit(&bars->s_full);
+          tc_commit(&bars->stage_empty[j & 1]);  // Q, dO and the statistics of step j
+          if (!more) tc_commit(&bars->o_final);
         }
         __syncwarp();
-        if (!wait_all(&bars->p_full, j & 1)) break;
-        // dV += P^T dO, dK += dS^T Q  (A from TMEM, B MN-major from the stage)
-        if (elect_one()) {
-          tc_fence_after();
-          issue_pv_ts_w<D, 128>(tmem + C::COL_ACC1, tmem + C::COL_S, desc_sw128(sDO, 128 * 128, 1024), j > 0);
-          issue_pv_ts_w<D, 128>(tmem + C::COL_ACC0, tmem + C::COL_DP, desc_sw128(sQ, 128 * 128, 1024), j > 0);
-          tc_commit(&bars->stage_empty[st]);
-          if (j + 1 == nsteps) tc_commit(&bars->o_final);
-        }
-        __syncwarp();
+        if (more) issue_s(j + 1, 1);
       }
       if (elect_one()) tc_commit(&bars->drain);
       __syncwarp();
@@ -306,32 +334,38 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dkdv_kernel(const __grid_cons
     const uint32_t tS = tmem + lane_off + C::COL_S, tDP = tmem + lane_off + C::COL_DP;
     const int off = a.Nk - a.Nq;
     bool ok = true;
-    for (int j = 0; j < nsteps; ++j) {
+    for (int j = 0; j < nsteps && ok; ++j) {
       const int st = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, abort_flag, a.timeout_ns) &&
-                                       mbar_wait(&bars->stage_full[st], (j >> 1) & 1, abort_flag, a.timeout_ns))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->stage_full[st], (j >> 1) & 1, abort_flag, a.timeout_ns))) {
         ok = false;
         break;
       }
-      tc_fence_after();
       const float* L2 = stat + st * 256;
       // visible query columns of this key row: q >= k - off (causal)
       const int lo = a.causal ? k - off - step_q0(j) : -1;
+      for (int h = 0; h < 2; ++h) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[h], j & 1, abort_flag, a.timeout_ns))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t s[32], dp[32], P[16], dS[16];
-        tmem_ld32(tS + 32 * cc, s);
-        tmem_ld32(tDP + 32 * cc, dp);
-        tmem_ld_wait(s);
-        tmem_ld_wait(dp);
-        bwd_chunk(s, dp, a.scale_log2, L2 + 32 * cc, L2 + 128 + 32 * cc, lo - 32 * cc, 31, P, dS);
-        tmem_st16(tS + 16 * cc, P);   // P^T over S^T columns already read
-        tmem_st16(tDP + 16 * cc, dS);
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c0 = 64 * h + 32 * cc;  // first query column of the chunk
+          uint32_t sv[32], dp[32], P[16], dS[16];
+          tmem_ld32(tS + c0, sv);
+          tmem_ld32(tDP + c0, dp);
+          tmem_ld_wait(sv);
+          tmem_ld_wait(dp);
+          bwd_chunk(sv, dp, a.scale_log2, L2 + c0, L2 + 128 + c0, lo - c0, 31, P, dS);
+          tmem_st16(tS + 64 * h + 16 * cc, P);  // packed over the half's columns already read
+          tmem_st16(tDP + 64 * h + 16 * cc, dS);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[h]);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full);
     }
     ok = __all_sync(0xffffffffu, ok);
     const bool have = nsteps > 0;
@@ -428,26 +462,48 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dq_kernel(const __grid_consta
     };
     if (nsteps > 0) {
       const Desc dq = desc_sw128(sQ, 16, 1024), ddo = desc_sw128(sDO, 16, 1024);
-      bool ok = wait_all(&bars->fixed_full, 0);
+      // halves of 64 keys: S_h = Q K_h^T, dP_h = dO V_h^T, then dQ += dS_h K_h
+      auto stage_k = [&](int j) { return sRing + (j & 1) * 2 * C::TILE_BYTES; };
+      auto issue_s = [&](int j, int h) {
+        const uint32_t sK = stage_k(j) + h * C::HALF_ROWS_BYTES, sV = sK + C::TILE_BYTES;
+        if (elect_one()) {
+          tc_fence_after();
+          issue_qk_rows<D, 64>(tmem + C::COL_S + 64 * h, dq, desc_sw128(sK, 16, 1024));
+          issue_qk_rows<D, 64>(tmem + C::COL_DP + 64 * h, ddo, desc_sw128(sV, 16, 1024));
+          tc_commit(&bars->s_full[h]);
+        }
+        __syncwarp();
+      };
+      auto issue_acc = [&](int j, int h) {
+        const uint32_t sK = stage_k(j) + h * C::HALF_ROWS_BYTES;
+        if (elect_one()) {
+          tc_fence_after();
+          issue_pv_ts_w<D, 64>(tmem + C::COL_ACC0, tmem + C::COL_S + 64 * h, desc_sw128(sK, 128 * 128, 1024),
+                               j > 0 || h > 0);
+        }
+        __syncwarp();
+      };
+      bool ok = wait_all(&bars->fixed_full, 0) && wait_all(&bars->stage_full[0], 0);
+      if (ok) {
+        issue_s(0, 0);
+        issue_s(0, 1);
+      }
       for (int j = 0; j < nsteps && ok; ++j) {
-        const int st = j & 1;
-        const uint32_t sK = sRing + st * 2 * C::TILE_BYTES, sV = sK + C::TILE_BYTES;
-        if (!wait_all(&bars->stage_full[st], (j >> 1) & 1)) break;
-        if (elect_one()) {  // S = Q K^T, dP = dO V^T
-          tc_fence_after();
-          issue_qk_w<D, 128>(tmem + C::COL_S, dq, desc_sw128(sK, 16, 1024));
-          issue_qk_w<D, 128>(tmem + C::COL_DP, ddo, desc_sw128(sV, 16, 1024));
-          tc_commit(&bars->s_full);
+        const bool more = j + 1 < nsteps;
+        if (!wait_all(&bars->p_full[0], j & 1)) break;
+        issue_acc(j, 0);
+        if (more) {
+          if (!wait_all(&bars->stage_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) break;
+          issue_s(j + 1, 0);
+        }
+        if (!wait_all(&bars->p_full[1], j & 1)) break;
+        issue_acc(j, 1);
+        if (elect_one()) {
+          tc_commit(&bars->stage_empty[j & 1]);
+          if (!more) tc_commit(&bars->o_final);
         }
         __syncwarp();
-        if (!wait_all(&bars->p_full, j & 1)) break;
-        if (elect_one()) {  // dQ += dS K
-          tc_fence_after();
-          issue_pv_ts_w<D, 128>(tmem + C::COL_ACC0, tmem + C::COL_S, desc_sw128(sK, 128 * 128, 1024), j > 0);
-          tc_commit(&bars->stage_empty[st]);
-          if (j + 1 == nsteps) tc_commit(&bars->o_final);
-        }
-        __syncwarp();
+        if (more) issue_s(j + 1, 1);
       }
       if (elect_one()) tc_commit(&bars->drain);
       __syncwarp();
@@ -469,29 +525,32 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dq_kernel(const __grid_consta
       dlv[i] = dl;
     }
     bool ok = true;
-    for (int j = 0; j < nsteps; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, abort_flag, a.timeout_ns))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+    for (int j = 0; j < nsteps && ok; ++j) {
       // visible key columns of this query row: key < Nk, and key <= q + off (causal)
       int hi = a.Nk - 1 - j * 128;
       if (a.causal) hi = min(hi, q + off - j * 128);
+      for (int h = 0; h < 2; ++h) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[h], j & 1, abort_flag, a.timeout_ns))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t s[32], dp[32], P[16], dS[16];
-        tmem_ld32(tS + 32 * cc, s);
-        tmem_ld32(tDP + 32 * cc, dp);
-        tmem_ld_wait(s);
-        tmem_ld_wait(dp);
-        bwd_chunk(s, dp, a.scale_log2, L2v, dlv, 0, hi - 32 * cc, P, dS);
-        tmem_st16(tS + 16 * cc, dS);  // dS over S columns already read
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c0 = 64 * h + 32 * cc;
+          uint32_t sv[32], dp[32], P[16], dS[16];
+          tmem_ld32(tS + c0, sv);
+          tmem_ld32(tDP + c0, dp);
+          tmem_ld_wait(sv);
+          tmem_ld_wait(dp);
+          bwd_chunk(sv, dp, a.scale_log2, L2v, dlv, 0, hi - c0, P, dS);
+          tmem_st16(tS + 64 * h + 16 * cc, dS);  // over the half's S columns already read
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[h]);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full);
     }
     ok = __all_sync(0xffffffffu, ok);
     const bool have = nsteps > 0;

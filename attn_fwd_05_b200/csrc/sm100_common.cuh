@@ -246,6 +246,18 @@ __device__ __forceinline__ void issue_qk_w(uint32_t s_tmem, Desc q, Desc k) {
              k.lo + (uint32_t)((((kk >> 2) * (BN * 128)) + (kk & 3) * 32) >> 4), k.hi, idesc, kk > 0 ? 1u : 0u);
 }
 
+// D(128 x N) = A B^T for 128-row tiles (chunk stride 128 x 128 bytes) of which B
+// contributes N rows from its descriptor base (a 64-row half of a tile, say).
+template <int D, int N>
+__device__ __forceinline__ void issue_qk_rows(uint32_t s_tmem, Desc a, Desc b) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, N, 0, 0);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (uint32_t)((((kk >> 2) * (128 * 128)) + (kk & 3) * 32) >> 4);
+    mma_ss_w(s_tmem, a.lo + off, a.hi, b.lo + off, b.hi, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
 template <int D, int BN>
 __device__ __forceinline__ void issue_pv_w(uint32_t o_tmem, Desc p, Desc v, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
