@@ -65,7 +65,8 @@ def parse():
     return p.parse_args()
 
 
-CSRC = ("attn_api.cu", "decode_sm100.cuh", "prefill_sm100.cuh", "sm100_common.cuh")
+CSRC = ("attn_api.cu", "backward_sm100.cuh", "decode_sm100.cuh", "fwd_fp8_sm100.cuh", "prefill_sm100.cuh",
+        "sm100_common.cuh")
 
 
 def csrc_digest() -> str:
@@ -521,7 +522,9 @@ def run_fp8(args, dist):
                    "l2": "L2 flushed between steps by writing a 256 MB buffer",
                    "parallelism": f"independent replicas x{dist.world} (no data-path collective)"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak,
+                     "traffic": profiled_traffic("attn_fwd_fp8_gqa_causal_2k.md")
+                     if args.workload == "gqa_causal_2k_fp8" else None,
                      "peak_source": f"2 x {peak_src} bf16_tflops (nominal e4m3 : bf16 dense ratio)",
                      "kernel": "attn_fwd_fp8_kernel", "flops_per_launch": flops, "median_ms": statistics.median(ms)},
         "gpu_launches": K, "clocks": clk,
