@@ -19,7 +19,8 @@
 //     scaled by 256 and rounded to e4m3 into shared memory; 256 = 2^8 is exact in e4m3,
 //     which keeps the largest probability exact, and pushes probabilities down to 2^-17
 //     above the format's smallest subnormal;
-//   * O = O_acc * sv / (256 l) in the epilogue, l the fp32 sum of the unrounded P.
+//   * O = O_acc * sv / l' in the epilogue, l' the fp32 sum of the unrounded 256 P (the
+//     factor 2^8 is added in the exponent: 2^(y + 8) = 256 2^y, exactly).
 #pragma once
 
 #include "sm100_common.cuh"
@@ -418,33 +419,49 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_fp8_kernel(const __grid_const
         // mask: keys past Nk, and past the diagonal when causal
         int lim = a.Nk - 1 - kb * 128;
         if (a.causal) lim = min(lim, khi - kb * 128);
+        // raw scores (units of the fp8 products); the mask only where the block needs it
         float s[128];
 #pragma unroll
-        for (int i = 0; i < 128; ++i) s[i] = (i > lim) ? -INFINITY : __uint_as_float(rs[i]) * c;
+        for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(rs[i]);
+        const bool masked = lim < 127;
+        if (masked) {
+#pragma unroll
+          for (int i = 0; i < 128; ++i) s[i] = (i > lim) ? -INFINITY : s[i];
+        }
         float x0 = max3(s[0], s[1], s[2]), x1 = max3(s[3], s[4], s[5]);
 #pragma unroll
         for (int i = 6; i < 126; i += 4) {
           x0 = max3(x0, s[i], s[i + 1]);
           x1 = max3(x1, s[i + 2], s[i + 3]);
         }
-        const float mx = max3(x0, x1, fmaxf(s[126], s[127]));
+        const float mx = max3(x0, x1, fmaxf(s[126], s[127])) * c;  // c > 0 commutes with the max
         float alpha = 1.0f;
         if (mx > m) {
           alpha = ex2(m - mx);
           m = mx;
         }
-        const float nmu = (m == -INFINITY) ? 0.0f : -m;
+        // p' = 256 p = 2^(s c - m + 8): the factor 2^8 rides in the exponent; l sums p'
+        const float nmu = (m == -INFINITY) ? 0.0f : 8.0f - m;
         uint32_t P[32];
         float a0 = 0.f, a1 = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2(s[4 * i] + nmu), p1 = ex2(s[4 * i + 1] + nmu);
-          const float p2 = ex2(s[4 * i + 2] + nmu), p3 = ex2(s[4 * i + 3] + nmu);
-          a0 += p0 + p1;
-          a1 += p2 + p3;
-          P[i] = pack_e4m3x4(p0 * 256.f, p1 * 256.f, p2 * 256.f, p3 * 256.f);
+          float y0, y1, y2, y3, p0, p1, p2, p3;
+          fma2(y0, y1, s[4 * i], s[4 * i + 1], c, c, nmu, nmu);
+          fma2(y2, y3, s[4 * i + 2], s[4 * i + 3], c, c, nmu, nmu);
+          if (!masked && (i & 3) == 3) {  // a quarter of the pairs on the FMA pipe, as in the bf16 kernel
+            exp2_fma2(p0, p1, y0, y1);
+          } else {
+            p0 = ex2(y0);
+            p1 = ex2(y1);
+          }
+          p2 = ex2(y2);
+          p3 = ex2(y3);
+          add2(a0, a1, p0, p1);
+          add2(a0, a1, p2, p3);
+          P[i] = pack_e4m3x4(p0, p1, p2, p3);
         }
-        l = l * alpha + (a0 + a1);
+        l = l * alpha + (a0 + a1);  // in units of 256
         if (!__all_sync(0xffffffffu,
                         k == 0 || mbar_wait(&bars->o_done[t], (k - 1) & 1, abort_flag, a.timeout_ns))) {
           fail = true;
@@ -487,7 +504,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_fp8_kernel(const __grid_const
       const bool valid = r < job.rows;
       const size_t row = bhq * (size_t)a.Nq + (size_t)(valid ? q : 0);
       const float sv = __ldg(&a.v_scale[(size_t)b * a.Hkv + kvh]);
-      const float inv = l > 0.f ? sv / (256.f * l) : 0.f;
+      const float inv = l > 0.f ? sv / l : 0.f;  // l already carries the factor 256
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t ro[32];
@@ -518,7 +535,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_fp8_kernel(const __grid_const
           }
         }
       }
-      if (valid && a.lse != nullptr) a.lse[row] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
+      if (valid && a.lse != nullptr) a.lse[row] = (l > 0.f) ? (m + log2f(l) - 8.0f) * kLn2 : -INFINITY;
     }
   }
 
