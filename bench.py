@@ -269,8 +269,6 @@ def oracle_prefill_sample(shape, q, k, v, seconds: float, max_heads=None):
     i = 0
     while i < len(heads):
         batch = heads[i:i + threads]
-        for b, h in batch:
-            pass
         qs = torch.stack([q[b, h] for b, h in batch])[None]
         ks = torch.stack([k[b, h // G] for b, h in batch])[None]
         vs = torch.stack([v[b, h // G] for b, h in batch])[None]
@@ -305,10 +303,62 @@ def oracle_decode_sample(dec, seconds: float):
 
 # ----------------------------------------------------------------------------- arms
 
+def run_reference_variant(args, dist):
+    """Reference arm of the backward and FP8 workloads: the fp64 backward oracle, or the
+    fp64 attention of the dequantized e4m3 inputs, on bounded samples of whole heads."""
+    import oracle
+    bwd = args.workload.endswith("_bwd")
+    name = args.workload[:-4]
+    shape = synth.WORKLOADS[name]
+    seed = synth.workload_seed(name)
+    q, k, v = synth.prefill_inputs(shape, seed)
+    scale = synth.default_scale(shape.d)
+    fwd_flops = counts.prefill_flops(shape.B, shape.Hq, shape.Nq, shape.Nk, shape.d, shape.causal)
+    per_step = max(0.5, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
+    if bwd:
+        do = synth.upstream_grad(shape, seed)
+        run = lambda: oracle_backward_sample(shape, (q, k, v), do, scale, 2.5 * fwd_flops, per_step)  # noqa: E731
+        metric, dtype = "attn bwd TFLOPS & % of BF16 tensor peak", "f64"
+    else:
+        q8, qs = oracle.block_quantize(q, 128)
+        k8, ks = oracle.block_quantize(k, 128)
+        v8, vs = oracle.block_quantize(v, shape.Nk)
+        qd, kd = torch.from_numpy(oracle.dequantize(q8, qs)), torch.from_numpy(oracle.dequantize(k8, ks))
+        vd = torch.from_numpy(oracle.dequantize(v8, vs, block=shape.Nk))
+        run = lambda: oracle_prefill_sample(shape, qd, kd, vd, per_step, max_heads=os.cpu_count())  # noqa: E731
+        metric, dtype = "attn fwd TFLOPS (e4m3 inputs) & % of FP8 tensor peak", "f64"
+    for _ in range(args.warmup):
+        run()
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(run()["value"])
+    total = time.perf_counter() - t0
+    value = statistics.mean(vals) if vals else 0.0
+    sample = ("per step: whole (batch, head) pairs of the fp64 backward oracle, one thread" if bwd else
+              f"per step: {os.cpu_count()} (batch, head) pairs of the fp64 oracle on the dequantized inputs")
+    line = {
+        "impl": "reference", "metric": metric, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+        "config": {"workload": args.workload,
+                   "prefill": {"B": shape.B, "Hq": shape.Hq, "Hkv": shape.Hkv, "Nq": shape.Nq, "Nk": shape.Nk,
+                               "d": shape.d, "causal": shape.causal},
+                   "parallelism": f"independent replicas x{args.gpus} (no data-path collective)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1 if bwd else os.cpu_count(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_reference(args, dist):
     """The oracle, as it stands, on the host cores, on the same config and metric."""
     if dist.rank != 0:
         return 0
+    if args.workload.endswith(("_bwd", "_fp8")):
+        return run_reference_variant(args, dist)
     shape = prefill_shape(args.workload)
     q, k, v = synth.prefill_inputs(shape, synth.workload_seed(
         "gqa_causal_2k" if args.workload == "serving_step" else args.workload))
