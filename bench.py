@@ -69,13 +69,25 @@ CSRC = ("attn_api.cu", "backward_sm100.cuh", "decode_sm100.cuh", "fwd_fp8_sm100.
         "sm100_common.cuh")
 
 
-def csrc_digest() -> str:
-    """sha256 prefix of the kernel sources without their comments and blank space, to match
+# the sources each committed ncu summary's kernel is built from (kernel header, shared
+# device helpers, host launch code)
+PROFILE_SOURCES = {
+    "attn_fwd_pingpong_gqa_causal_2k.md": ("attn_api.cu", "prefill_sm100.cuh", "sm100_common.cuh"),
+    "attn_fwd_pingpong_gqa_causal_16k.md": ("attn_api.cu", "prefill_sm100.cuh", "sm100_common.cuh"),
+    "attn_fwd_single_peaked_mha_d256.md": ("attn_api.cu", "prefill_sm100.cuh", "sm100_common.cuh"),
+    "attn_decode_split_paged_decode.md": ("attn_api.cu", "decode_sm100.cuh", "sm100_common.cuh"),
+    "attn_bwd_gqa_causal_2k.md": ("attn_api.cu", "backward_sm100.cuh", "sm100_common.cuh"),
+    "attn_fwd_fp8_gqa_causal_2k.md": ("attn_api.cu", "fwd_fp8_sm100.cuh", "sm100_common.cuh"),
+}
+
+
+def csrc_digest(files=CSRC) -> str:
+    """sha256 prefix of kernel sources without their comments and blank space, to match
     against the committed ncu summaries (a comment edit does not change the kernels)."""
     import hashlib
     import re
     h = hashlib.sha256()
-    for name in CSRC:
+    for name in files:
         with open(os.path.join(ROOT, "attn_fwd_05_b200", "csrc", name)) as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
@@ -104,7 +116,7 @@ def profiled_traffic(profile: str, scale: float = 1.0):
     import re
     m_sha = re.search(r"csrc sha256 prefix `([0-9a-f]+)`", text)
     m_b = re.search(r"traffic_bytes_per_launch: (\d+)", text)
-    if not (m_sha and m_b) or m_sha.group(1) != csrc_digest():
+    if not (m_sha and m_b) or m_sha.group(1) != csrc_digest(PROFILE_SOURCES.get(profile, CSRC)):
         return None
     return int(m_b.group(1)) * scale
 
@@ -463,7 +475,8 @@ def run_backward(args, dist):
                    "l2": "L2 flushed between steps by writing a 256 MB buffer",
                    "parallelism": f"independent replicas x{dist.world} (no data-path collective)"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                     "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": profiled_traffic("attn_bwd_gqa_causal_2k.md") if name == "gqa_causal_2k" else None,
                      "peak_source": f"{peak_src} bf16_tflops (burst cuBLAS)",
                      "kernel": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel + attn_bwd_delta_kernel (one call)",
                      "flops_per_launch": flops, "median_ms": statistics.median(ms)},

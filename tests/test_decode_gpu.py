@@ -43,7 +43,9 @@ CASES = [
     ([3000, 1024, 1025, 2048], 8, 1, 128, 16),     # chunk edges, MQA with 8 query heads
     ([700, 33, 64], 4, 4, 64, 32),                 # d=64, 32-token pages, MHA
     ([513, 130], 4, 2, 256, 64),                   # d=256, 64-token pages
-    ([900, 77], 32, 2, 128, 16),                   # 16 query heads per KV head, two head groups
+    ([900, 77], 32, 2, 128, 16),                   # 16 query heads per KV head: one full head group
+    ([1300, 5], 40, 2, 128, 16),                   # 20 per KV head: head groups of 16 and 4 rows
+    ([2100, 600], 64, 1, 128, 16),                 # 64 per KV head (MQA): four head groups
     ([2500], 3, 1, 128, 16),                       # odd group
 ]
 
