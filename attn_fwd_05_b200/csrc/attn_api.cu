@@ -292,6 +292,8 @@ attn_status fwd_common(const void* q, const void* k, const void* v, void* o, int
   if (!encode_3d(&a.tm_q, q, d, Nq, (uint64_t)B * Hq, 128) || !encode_3d(&a.tm_k, k, d, Nk, (uint64_t)B * Hkv, bn) ||
       !encode_3d(&a.tm_v, v, d, Nk, (uint64_t)B * Hkv, bn))
     return ATTN_ERR_CUDA;
+  // bf16 O of the two-tile kernel leaves through TMA stores of 32-row boxes
+  if (!o_f32 && d <= 128 && !encode_3d(&a.tm_o, o, d, Nq, (uint64_t)B * Hq, 32)) return ATTN_ERR_CUDA;
   a.o = o;
   a.lse = lse;
   a.B = B;

@@ -44,6 +44,7 @@ struct FwdArgs {
   CUtensorMap tm_q;  // [B*Hq, Nq, d] bf16, box {64, 128, 1}
   CUtensorMap tm_k;  // [B*Hkv, Nk, d] bf16, box {64, BN, 1}
   CUtensorMap tm_v;
+  CUtensorMap tm_o;  // bf16 O [B*Hq, Nq, d], box {64, 32, 1}: stores of the two-tile kernel (d <= 128)
   void* o;
   float* lse;
   int B, Hq, Hkv, Nq, Nk;
@@ -407,6 +408,37 @@ __device__ __forceinline__ void store_cols(const FwdArgs& a, uint32_t o_taddr, b
   }
 }
 
+// Row r of O / l as bf16 into a 128-row tile in the P layout (128-byte swizzled
+// 64-column chunks), from where TMA writes it to global memory: one 16-byte store per
+// 8 columns, conflict-free like the P stores, instead of 32 rows' worth of scattered
+// global stores per warp instruction.
+template <int D>
+__device__ __forceinline__ void stage_o_row(uint32_t tile, int r, uint32_t o_taddr, bool have_o, float l) {
+  const float inv = l > 0.f ? 1.0f / l : 0.f;
+  const uint32_t row = tile + (uint32_t)r * 128u;
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t v[32];
+    if (have_o) {
+      tmem_ld32(o_taddr + c * 32, v);
+      tmem_ld_wait(v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        w[i] = pack_bf16x2(__uint_as_float(v[8 * j + 2 * i]) * inv, __uint_as_float(v[8 * j + 2 * i + 1]) * inv);
+      const int g = (c & 1) * 4 + j;  // 16-byte granule within the 64-column chunk c / 2
+      st_shared_v4(row + (uint32_t)((c >> 1) * (128 * 128)) + (uint32_t)((g ^ (r & 7)) << 4), w[0], w[1], w[2],
+                   w[3]);
+    }
+  }
+}
+
 // Work unit u of the two-tile kernel: two 128-row Q tiles and the KV head they read.
 // Causal: heaviest q-tiles first (longest-processing-time order).  Otherwise all units
 // weigh about the same; consecutive units share a head so that the K/V tiles streamed at
@@ -695,6 +727,16 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
     int k = 0;         // this tile's visits over all units (barrier phases)
     int nfin = 0;      // units in which this tile had visits (o_final phases)
     bool fail = false;  // a wait gave up (the warp decides as one)
+    // this warp's last O store (bf16 O) still reads its rows of P_t: lane 0 waits for
+    // that before the rows are written again
+    bool store_pending = false;
+    auto settle_store = [&]() {
+      if (store_pending) {
+        if (lane == 0) bulk_wait_read();
+        __syncwarp();
+        store_pending = false;
+      }
+    };
     for (int rd = 0; rd * (int)gridDim.x < a.n_units && !fail; ++rd) {
       const int u = snake_unit(rd);
       if (u >= a.n_units) continue;
@@ -741,6 +783,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
           fail = true;
           break;
         }
+        settle_store();
         store_p_row<BN / 2>(p_tile, r, P);
         fence_proxy_async_smem();
         if (kl > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
@@ -769,9 +812,28 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
       }
       const bool valid = r < job.rows;
       const size_t row = ((size_t)b * a.Hq + job.hq) * (size_t)a.Nq + (size_t)(valid ? q : 0);
-      store_cols<D>(a, o_addr, have_o, valid, row * D, l);
+      if (a.o_f32) {
+        store_cols<D>(a, o_addr, have_o, valid, row * D, l);
+      } else if (job.rows > quad * 32) {  // the warp has valid rows (warp-uniform)
+        // P_t is free (the tile's last P V of the unit is done, or it had none): stage
+        // this warp's 32 rows there and store them with TMA (rows past Nq are clipped)
+        settle_store();
+        stage_o_row<D>(p_tile, r, o_addr, have_o, l);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_store_3d(&a.tm_o, p_tile + (uint32_t)(c * (128 * 128) + quad * 32 * 128), c * 64, job.q0 + quad * 32,
+                         b * a.Hq + job.hq);
+          bulk_commit();
+        }
+        store_pending = true;
+      }
       if (valid && a.lse != nullptr) a.lse[row] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
     }
+    if (lane == 0) bulk_wait_all();  // this warp's O stores are done before the CTA exits
+    __syncwarp();
   }
 
   tc_fence_before();
