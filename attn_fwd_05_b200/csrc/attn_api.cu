@@ -380,6 +380,7 @@ attn_status attn_fwd_fp8(const void* q8, const float* q_scale, const void* k8, c
   if (!encode_3d_u8(&a.tm_q, q8, Nq, (uint64_t)B * Hq) || !encode_3d_u8(&a.tm_k, k8, Nk, (uint64_t)B * Hkv) ||
       !encode_3d_u8(&a.tm_v, v8, Nk, (uint64_t)B * Hkv))
     return ATTN_ERR_CUDA;
+  if (!o_f32 && !encode_3d(&a.tm_o, o, 128, Nq, (uint64_t)B * Hq, 32)) return ATTN_ERR_CUDA;
   a.q_scale = q_scale;
   a.k_scale = k_scale;
   a.v_scale = v_scale;

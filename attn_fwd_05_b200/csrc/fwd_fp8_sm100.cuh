@@ -31,6 +31,7 @@ struct Fp8Args {
   CUtensorMap tm_q;  // [B*Hq, Nq, 128] uint8 (e4m3), box {128, 128, 1}
   CUtensorMap tm_k;  // [B*Hkv, Nk, 128]
   CUtensorMap tm_v;
+  CUtensorMap tm_o;      // bf16 O [B*Hq, Nq, 128], box {64, 32, 1} (unused for fp32 O)
   const float* q_scale;  // [B*Hq, ceil(Nq/128)]
   const float* k_scale;  // [B*Hkv, ceil(Nk/128)]
   const float* v_scale;  // [B*Hkv]
@@ -134,11 +135,15 @@ struct Fp8Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_P = 2 * TILE;
   static constexpr int OFF_KV = 4 * TILE;
-  static constexpr int OFF_BAR = OFF_KV + NSTAGE * TILE;
+  // bf16 O of a tile leaves through TMA stores of two 64-column chunks, staged in the
+  // tile's P buffer and in one more 16 KB buffer per tile
+  static constexpr int OFF_X = OFF_KV + NSTAGE * TILE;
+  static constexpr int OFF_BAR = OFF_X + 2 * TILE;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + 1 KB alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 384;
 };
+static_assert(Fp8Cfg::SMEM <= 227 * 1024, "shared memory");
 
 struct Fp8Bars {
   uint64_t q_full[2];
@@ -387,8 +392,18 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_fp8_kernel(const __grid_const
     const uint32_t s_addr = tmem + lane_off + (t ? C::COL_S1 : C::COL_S0);
     const uint32_t o_addr = tmem + lane_off + (t ? C::COL_O1 : C::COL_O0);
     const uint32_t p_row = sP + t * C::TILE + (uint32_t)r * 128u;
+    const uint32_t x_tile = smem_u32(smem + C::OFF_X) + t * C::TILE;
     int k = 0, nfin = 0;
     bool fail = false;
+    // this warp's last O store still reads its rows of the staging buffers (P_t, X_t)
+    bool store_pending = false;
+    auto settle_store = [&]() {
+      if (store_pending) {
+        if (lane == 0) bulk_wait_read();
+        __syncwarp();
+        store_pending = false;
+      }
+    };
     for (int rd = 0; rd * (int)gridDim.x < a.n_units && !fail; ++rd) {
       const int u = snake_unit(rd);
       if (u >= a.n_units) continue;
@@ -467,21 +482,27 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_fp8_kernel(const __grid_const
           fail = true;
           break;
         }
+        settle_store();
 #pragma unroll
         for (int g = 0; g < 8; ++g)  // 16-byte granule g (keys 16g..16g+15) at g ^ (r % 8)
           st_shared_v4(p_row + (uint32_t)((g ^ (r & 7)) << 4), P[4 * g], P[4 * g + 1], P[4 * g + 2], P[4 * g + 3]);
         fence_proxy_async_smem();
         if (kl > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
           tc_fence_after();
+          uint32_t ro[128];  // one TMEM round trip for the whole row
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t ro[32];
-            tmem_ld32(o_addr + 32 * j, ro);
-            tmem_ld_wait(ro);
+          for (int j = 0; j < 4; ++j) tmem_ld32(o_addr + 32 * j, *reinterpret_cast<uint32_t(*)[32]>(&ro[32 * j]));
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) * alpha);
-            tmem_st32(o_addr + 32 * j, ro);
+          for (int j = 0; j < 4; ++j) tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&ro[32 * j]));
+#pragma unroll
+          for (int i = 0; i < 128; i += 2) {
+            float u0 = __uint_as_float(ro[i]), u1 = __uint_as_float(ro[i + 1]);
+            mul2(u0, u1, alpha, alpha);
+            ro[i] = __float_as_uint(u0);
+            ro[i + 1] = __float_as_uint(u1);
           }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) tmem_st32(o_addr + 32 * j, *reinterpret_cast<uint32_t(*)[32]>(&ro[32 * j]));
           tmem_st_wait();
         }
         tc_fence_before();
@@ -505,6 +526,44 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_fp8_kernel(const __grid_const
       const size_t row = bhq * (size_t)a.Nq + (size_t)(valid ? q : 0);
       const float sv = __ldg(&a.v_scale[(size_t)b * a.Hkv + kvh]);
       const float inv = l > 0.f ? sv / l : 0.f;  // l already carries the factor 256
+      if (!a.o_f32) {
+        if (job.rows > quad * 32) {  // the warp has valid rows (warp-uniform)
+          // P_t is free (the tile's last P V of the unit is done, or it had none): this
+          // warp's 32 rows of O go to P_t (columns 0-63) and X_t (64-127), swizzled like
+          // P, and TMA stores them (rows past Nq are clipped)
+          settle_store();
+          uint32_t ro[128];
+          if (have_o) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tmem_ld32(o_addr + 32 * j, *reinterpret_cast<uint32_t(*)[32]>(&ro[32 * j]));
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&ro[32 * j]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 128; ++i) ro[i] = 0u;
+          }
+          const uint32_t xrow = x_tile + (uint32_t)r * 128u;
+#pragma unroll
+          for (int g = 0; g < 16; ++g) {  // 16-byte granule: 8 columns
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              w[i] = pack_bf16x2(__uint_as_float(ro[8 * g + 2 * i]) * inv, __uint_as_float(ro[8 * g + 2 * i + 1]) * inv);
+            st_shared_v4((g < 8 ? p_row : xrow) + (uint32_t)(((g & 7) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t off = (uint32_t)(quad * 32 * 128);
+            tma_store_3d(&a.tm_o, sP + t * C::TILE + off, 0, job.q0 + quad * 32, (int)bhq);
+            tma_store_3d(&a.tm_o, x_tile + off, 64, job.q0 + quad * 32, (int)bhq);
+            bulk_commit();
+          }
+          store_pending = true;
+        }
+        if (valid && a.lse != nullptr) a.lse[row] = (l > 0.f) ? (m + log2f(l) - 8.0f) * kLn2 : -INFINITY;
+        continue;
+      }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t ro[32];
@@ -537,6 +596,8 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_fp8_kernel(const __grid_const
       }
       if (valid && a.lse != nullptr) a.lse[row] = (l > 0.f) ? (m + log2f(l) - 8.0f) * kLn2 : -INFINITY;
     }
+    if (lane == 0) bulk_wait_all();  // this warp's O stores are done before the CTA exits
+    __syncwarp();
   }
 
   tc_fence_before();

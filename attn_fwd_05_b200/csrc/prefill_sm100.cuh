@@ -352,22 +352,23 @@ __device__ __forceinline__ float load_scores(uint32_t s_taddr, bool masked, int 
   return max3(x0, x1, fmaxf(s[NCOL - 2], s[NCOL - 1])) * sl2;
 }
 
+// All NC columns are loaded before the one wait: one TMEM round trip, not NC / 32.
 template <int NC>
 __device__ __forceinline__ void rescale_cols(uint32_t o_taddr, float alpha) {
+  uint32_t r[NC];
 #pragma unroll
-  for (int c = 0; c < NC / 32; ++c) {
-    uint32_t r[32];
-    tmem_ld32(o_taddr + c * 32, r);
-    tmem_ld_wait(r);
+  for (int c = 0; c < NC / 32; ++c) tmem_ld32(o_taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-      float u0 = __uint_as_float(r[i]), u1 = __uint_as_float(r[i + 1]);
-      mul2(u0, u1, alpha, alpha);
-      r[i] = __float_as_uint(u0);
-      r[i + 1] = __float_as_uint(u1);
-    }
-    tmem_st32(o_taddr + c * 32, r);
+  for (int c = 0; c < NC / 32; ++c) tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+#pragma unroll
+  for (int i = 0; i < NC; i += 2) {
+    float u0 = __uint_as_float(r[i]), u1 = __uint_as_float(r[i + 1]);
+    mul2(u0, u1, alpha, alpha);
+    r[i] = __float_as_uint(u0);
+    r[i + 1] = __float_as_uint(u1);
   }
+#pragma unroll
+  for (int c = 0; c < NC / 32; ++c) tmem_st32(o_taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
 }
 
 // Epilogue for NC columns of one row: O / l to global (bf16 or fp32).
@@ -416,16 +417,19 @@ template <int D>
 __device__ __forceinline__ void stage_o_row(uint32_t tile, int r, uint32_t o_taddr, bool have_o, float l) {
   const float inv = l > 0.f ? 1.0f / l : 0.f;
   const uint32_t row = tile + (uint32_t)r * 128u;
+  uint32_t o[D];
+  if (have_o) {
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) tmem_ld32(o_taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32 * c]));
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&o[32 * c]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < D; ++i) o[i] = 0u;
+  }
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {
-    uint32_t v[32];
-    if (have_o) {
-      tmem_ld32(o_taddr + c * 32, v);
-      tmem_ld_wait(v);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = 0u;
-    }
+    const uint32_t* v = o + 32 * c;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       uint32_t w[4];
