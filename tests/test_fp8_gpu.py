@@ -50,11 +50,11 @@ def quantized_inputs(B, Hq, Hkv, Nq, Nk, seed):
     return (q8, qs, k8, ks, v8, vs[..., 0])
 
 
-def run_fp8(inp, causal, scale):
+def run_fp8(inp, causal, scale, out_dtype=torch.float32):
     dev = torch.device("cuda:0")
     q8, qs, k8, ks, v8, vs = (torch.from_numpy(np.ascontiguousarray(t)).to(dev) for t in inp)
     B, Hq, Nq, d = q8.shape
-    o = torch.empty((B, Hq, Nq, d), dtype=torch.float32, device=dev)
+    o = torch.empty((B, Hq, Nq, d), dtype=out_dtype, device=dev)
     lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
     ab.attn_fwd_fp8(q8, qs, k8, ks, v8, vs, o, lse, causal, scale)
     st = ab.attn_get_device_status()
@@ -109,6 +109,19 @@ def test_fp8_end_to_end_with_gpu_quantizer(cuda_device):
     o2, _ = run_fp8(ref, True, 1 / math.sqrt(128))
     # bf16 output of the same kernel: within half a bf16 unit of the fp32 output
     assert np.all(np.abs(o.double().cpu().numpy() - o2) <= np.abs(o2) * 2.0 ** -8 + 1e-6)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk,causal", [(1, 3, 1, 333, 333, True), (1, 2, 2, 33, 200, False),
+                                                   (2, 4, 2, 1, 129, True)])
+def test_fp8_bf16_store_equals_rounded_fp32_output(B, Hq, Hkv, Nq, Nk, causal, cuda_device):
+    # bf16 O leaves through staged tensor stores, fp32 O through direct stores
+    inp = quantized_inputs(B, Hq, Hkv, Nq, Nk, seed=900 + Nq)
+    scale = 1.0 / math.sqrt(128)
+    o32, l32 = run_fp8(inp, causal, scale)
+    o16, l16 = run_fp8(inp, causal, scale, out_dtype=torch.bfloat16)
+    rounded = torch.from_numpy(o32).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(o16, rounded)
+    assert np.array_equal(l16, l32)
 
 
 def test_fp8_rejects_other_head_dims(cuda_device):

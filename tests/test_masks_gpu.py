@@ -127,6 +127,17 @@ def test_all_zero_map_gives_zero_and_minus_inf(d, cuda_device):
     assert np.all(o == 0) and np.all(np.isneginf(lse))
 
 
+@pytest.mark.parametrize("Nq,Nk,d,window", [(333, 333, 128, 100), (45, 300, 64, 17)])
+def test_window_bf16_store_equals_rounded_fp32_output(Nq, Nk, d, window, cuda_device):
+    q, k, v = inputs(1, 4, 2, Nq, Nk, d, seed=23 + Nq)
+    scale = 1.0 / math.sqrt(d)
+    o32, l32 = run_masked(q, k, v, True, scale, window=window, out_dtype=torch.float32)
+    o16, l16 = run_masked(q, k, v, True, scale, window=window, out_dtype=torch.bfloat16)
+    rounded = torch.from_numpy(np.asarray(o32, dtype=np.float64)).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(np.asarray(o16, dtype=np.float64), rounded)
+    assert np.array_equal(l16, l32)
+
+
 def test_bad_masked_arguments_raise(cuda_device):
     q, k, v = inputs(1, 2, 2, 128, 128, 64, seed=1)
     dev = torch.device("cuda:0")

@@ -136,6 +136,25 @@ def test_bf16_output_is_rounded_fp32_output(cuda_device):
     assert np.array_equal(o16, rounded)
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk,d,causal", [
+    (1, 2, 2, 1, 77, 128, False),    # one row: a single valid row in the first warp's 32-row box
+    (1, 2, 2, 33, 300, 128, True),   # the second warp of the tile holds one valid row
+    (1, 3, 1, 333, 333, 128, True),  # odd group: q-tile pairs of one head, the last tile past Nq
+    (2, 4, 2, 257, 257, 64, True),   # d = 64: one 64-column box per warp
+    (1, 4, 4, 97, 130, 64, False),
+])
+def test_bf16_store_equals_rounded_fp32_output(B, Hq, Hkv, Nq, Nk, d, causal, cuda_device):
+    # bf16 O leaves through staged tensor stores, fp32 O through direct stores: the same
+    # accumulator and normaliser, so bf16 must be exactly the rounded fp32 output
+    q, k, v = inputs(B, Hq, Hkv, Nq, Nk, d, seed=17 + Nq, causal=causal)
+    scale = 1.0 / math.sqrt(d)
+    o32, l32 = run_prefill(q, k, v, causal, scale, out_dtype=torch.float32)
+    o16, l16 = run_prefill(q, k, v, causal, scale, out_dtype=torch.bfloat16)
+    rounded = torch.from_numpy(o32).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(o16, rounded)
+    assert np.array_equal(l16, l32)
+
+
 def test_watchdog_latches_timeout_and_device_stays_usable(cuda_device):
     assert ab.attn_get_device_status() == 0
     ab.attn_debug_watchdog(20_000_000)  # 20 ms on a barrier nothing completes
