@@ -194,6 +194,10 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Nq);
  *               16-byte aligned, owned by the caller (ATTN_ERR_WORKSPACE if too small).
  * Alignment: q, k, v, o, dout, dq, dk, dv 16-byte aligned.  A row with no visible key
  * (lse = -inf) gets zero gradient.  Nq = 0 writes dk = dv = 0; Nk = 0 writes dq = 0.
+ * Streams: the call is ordered on `stream` like any other: its dQ kernel runs on a
+ * library-owned stream that waits for the Delta pass enqueued on `stream`, and `stream`
+ * waits for the dQ kernel before anything enqueued after the call (an event fork and
+ * join, which CUDA graph capture records as such).
  */
 attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                      const float* lse, float* dq, float* dk, float* dv, int B, int Hq, int Hkv,
