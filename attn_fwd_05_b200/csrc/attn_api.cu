@@ -195,14 +195,14 @@ attn_status launch_bwd(attn::BwdArgs& a, const void* o, const void* dout, float*
   std::lock_guard<std::mutex> g(side_mutex());
   SideStream* side = side_stream();
   if (side != nullptr && cudaEventRecord(side->fork, st) != cudaSuccess) return ATTN_ERR_CUDA;
-  kkv<<<(unsigned)gkv, 256, C::SMEM, st>>>(a);
+  kkv<<<(unsigned)gkv, C::THREADS, C::SMEM, st>>>(a);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   if (side == nullptr) {
-    kq<<<(unsigned)gq, 256, C::SMEM, st>>>(a);
+    kq<<<(unsigned)gq, C::THREADS, C::SMEM, st>>>(a);
     return launch_status();
   }
   if (cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess) return ATTN_ERR_CUDA;
-  kq<<<(unsigned)gq, 256, C::SMEM, side->stream>>>(a);
+  kq<<<(unsigned)gq, C::THREADS, C::SMEM, side->stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   if (cudaEventRecord(side->join, side->stream) != cudaSuccess || cudaStreamWaitEvent(st, side->join, 0) != cudaSuccess)
     return ATTN_ERR_CUDA;

@@ -123,6 +123,29 @@ __device__ __forceinline__ void store_acc_row(uint32_t taddr, bool have, bool va
   }
 }
 
+// Columns [C0, C0 + NC) of this thread's accumulator row, as store_acc_row.
+template <int C0, int NC>
+__device__ __forceinline__ void store_acc_cols(uint32_t taddr, bool have, bool valid, float mul, float* dst) {
+#pragma unroll
+  for (int c = C0 / 32; c < (C0 + NC) / 32; ++c) {
+    uint32_t r[32];
+    if (have) {
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait(r);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) r[i] = 0u;
+    }
+    if (valid) {
+      float4* out = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        out[i] = make_float4(__uint_as_float(r[4 * i]) * mul, __uint_as_float(r[4 * i + 1]) * mul,
+                             __uint_as_float(r[4 * i + 2]) * mul, __uint_as_float(r[4 * i + 3]) * mul);
+    }
+  }
+}
+
 struct BwdBars {
   uint64_t fixed_full;  // the CTA's own tiles (K and V, or Q and dO) have landed
   uint64_t stage_full[2];
@@ -137,6 +160,9 @@ struct BwdBars {
 
 template <int D>
 struct BwdCfg {
+  // warp 0 TMA, 1 MMA, 2-3 statistics (dK/dV kernel), 4-7 and 8-11 the elementwise pass
+  // of query (dK/dV) or key (dQ) half 0 and half 1 of each step
+  static constexpr int THREADS = 384;
   static constexpr int T = 128;  // rows of every tile
   static constexpr int TILE_BYTES = T * D * 2;
   static constexpr int OFF_FIXED = 0;                       // two tiles
@@ -178,7 +204,7 @@ __device__ __forceinline__ int kv_qt_lo(const BwdArgs& a, int kt) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(256, 1) attn_bwd_dkdv_kernel(const __grid_constant__ BwdArgs a) {
+__global__ void __launch_bounds__(384, 1) attn_bwd_dkdv_kernel(const __grid_constant__ BwdArgs a) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -326,7 +352,9 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dkdv_kernel(const __grid_cons
       mbar_wait(&bars->drain, 0, abort_flag, a.timeout_ns, false);
     }
   } else {
-    // ================= warps 4-7: one key row per thread
+    // ================= warps 4-7 (half 0) and 8-11 (half 1): one key row per thread, the
+    // half's 64 query columns of every step
+    const int h = warp >= 8 ? 1 : 0;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int k = k0 + r;
@@ -343,29 +371,27 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dkdv_kernel(const __grid_cons
       const float* L2 = stat + st * 256;
       // visible query columns of this key row: q >= k - off (causal)
       const int lo = a.causal ? k - off - step_q0(j) : -1;
-      for (int h = 0; h < 2; ++h) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[h], j & 1, abort_flag, a.timeout_ns))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c0 = 64 * h + 32 * cc;  // first query column of the chunk
-          uint32_t sv[32], dp[32], P[16], dS[16];
-          tmem_ld32(tS + c0, sv);
-          tmem_ld32(tDP + c0, dp);
-          tmem_ld_wait(sv);
-          tmem_ld_wait(dp);
-          bwd_chunk(sv, dp, a.scale_log2, L2 + c0, L2 + 128 + c0, lo - c0, 31, P, dS);
-          tmem_st16(tS + 64 * h + 16 * cc, P);  // packed over the half's columns already read
-          tmem_st16(tDP + 64 * h + 16 * cc, dS);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_full[h]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[h], j & 1, abort_flag, a.timeout_ns))) {
+        ok = false;
+        break;
       }
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c0 = 64 * h + 32 * cc;  // first query column of the chunk
+        uint32_t sv[32], dp[32], P[16], dS[16];
+        tmem_ld32(tS + c0, sv);
+        tmem_ld32(tDP + c0, dp);
+        tmem_ld_wait(sv);
+        tmem_ld_wait(dp);
+        bwd_chunk(sv, dp, a.scale_log2, L2 + c0, L2 + 128 + c0, lo - c0, 31, P, dS);
+        tmem_st16(tS + 64 * h + 16 * cc, P);  // packed over the half's columns already read
+        tmem_st16(tDP + 64 * h + 16 * cc, dS);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full[h]);
     }
     ok = __all_sync(0xffffffffu, ok);
     const bool have = nsteps > 0;
@@ -373,11 +399,13 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dkdv_kernel(const __grid_cons
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_final, 0, abort_flag, a.timeout_ns));
       tc_fence_after();
     }
-    if (ok) {
+    if (ok) {  // half 0's warps write dK, half 1's dV
       const bool valid = k < a.Nk;
       const size_t row = ((size_t)bkv * a.Nk + (valid ? k : 0)) * D;
-      store_acc_row<D>(tmem + lane_off + C::COL_ACC0, have, valid, a.scale, a.dk + row);
-      store_acc_row<D>(tmem + lane_off + C::COL_ACC1, have, valid, 1.0f, a.dv + row);
+      if (h == 0)
+        store_acc_row<D>(tmem + lane_off + C::COL_ACC0, have, valid, a.scale, a.dk + row);
+      else
+        store_acc_row<D>(tmem + lane_off + C::COL_ACC1, have, valid, 1.0f, a.dv + row);
     }
   }
 
@@ -392,7 +420,7 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dkdv_kernel(const __grid_cons
 // ---------------------------------------------------------------------------- dQ
 
 template <int D>
-__global__ void __launch_bounds__(256, 1) attn_bwd_dq_kernel(const __grid_constant__ BwdArgs a) {
+__global__ void __launch_bounds__(384, 1) attn_bwd_dq_kernel(const __grid_constant__ BwdArgs a) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -510,7 +538,9 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dq_kernel(const __grid_consta
       mbar_wait(&bars->drain, 0, abort_flag, a.timeout_ns, false);
     }
   } else if (warp >= 4) {
-    // ================= one query row per thread
+    // ================= warps 4-7 (half 0) and 8-11 (half 1): one query row per thread,
+    // the half's 64 key columns of every step
+    const int h = warp >= 8 ? 1 : 0;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int q = q0 + r;
@@ -529,28 +559,26 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dq_kernel(const __grid_consta
       // visible key columns of this query row: key < Nk, and key <= q + off (causal)
       int hi = a.Nk - 1 - j * 128;
       if (a.causal) hi = min(hi, q + off - j * 128);
-      for (int h = 0; h < 2; ++h) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[h], j & 1, abort_flag, a.timeout_ns))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c0 = 64 * h + 32 * cc;
-          uint32_t sv[32], dp[32], P[16], dS[16];
-          tmem_ld32(tS + c0, sv);
-          tmem_ld32(tDP + c0, dp);
-          tmem_ld_wait(sv);
-          tmem_ld_wait(dp);
-          bwd_chunk(sv, dp, a.scale_log2, L2v, dlv, 0, hi - c0, P, dS);
-          tmem_st16(tS + 64 * h + 16 * cc, dS);  // over the half's S columns already read
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_full[h]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[h], j & 1, abort_flag, a.timeout_ns))) {
+        ok = false;
+        break;
       }
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c0 = 64 * h + 32 * cc;
+        uint32_t sv[32], dp[32], P[16], dS[16];
+        tmem_ld32(tS + c0, sv);
+        tmem_ld32(tDP + c0, dp);
+        tmem_ld_wait(sv);
+        tmem_ld_wait(dp);
+        bwd_chunk(sv, dp, a.scale_log2, L2v, dlv, 0, hi - c0, P, dS);
+        tmem_st16(tS + 64 * h + 16 * cc, dS);  // over the half's S columns already read
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full[h]);
     }
     ok = __all_sync(0xffffffffu, ok);
     const bool have = nsteps > 0;
@@ -558,10 +586,13 @@ __global__ void __launch_bounds__(256, 1) attn_bwd_dq_kernel(const __grid_consta
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_final, 0, abort_flag, a.timeout_ns));
       tc_fence_after();
     }
-    if (ok) {
+    if (ok) {  // each half's warps write half of the row's columns
       const bool valid = q < a.Nq;
-      store_acc_row<D>(tmem + lane_off + C::COL_ACC0, have, valid, a.scale,
-                       a.dq + ((size_t)bh * a.Nq + (valid ? q : 0)) * D);
+      float* dst = a.dq + ((size_t)bh * a.Nq + (valid ? q : 0)) * D;
+      if (h == 0)
+        store_acc_cols<0, D / 2>(tmem + lane_off + C::COL_ACC0, have, valid, a.scale, dst);
+      else
+        store_acc_cols<D / 2, D / 2>(tmem + lane_off + C::COL_ACC0, have, valid, a.scale, dst);
     }
   }
 
