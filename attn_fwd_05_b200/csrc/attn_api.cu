@@ -57,6 +57,21 @@ bool encode_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows
   return r == CUDA_SUCCESS;
 }
 
+// fp32 tensors [outer, rows, inner] with {32, 32, 1} boxes (128 bytes a row) and the
+// 128-byte swizzle: the backward's gradient stores.
+bool encode_3d_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {inner, rows, outer};
+  cuuint64_t strides[2] = {inner * 4, rows * inner * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // e4m3 tensors [outer, rows, 128 bytes]: one 128-byte swizzled row per token.
 bool encode_3d_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t outer) {
   EncodeTiledFn fn = encode_fn();
@@ -500,7 +515,9 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
   attn::BwdArgs a;
   std::memset(&a, 0, sizeof(a));
   if (!encode_3d(&a.tm_q, q, d, Nq, (uint64_t)B * Hq, 128) || !encode_3d(&a.tm_do, dout, d, Nq, (uint64_t)B * Hq, 128) ||
-      !encode_3d(&a.tm_k, k, d, Nk, (uint64_t)B * Hkv, 128) || !encode_3d(&a.tm_v, v, d, Nk, (uint64_t)B * Hkv, 128))
+      !encode_3d(&a.tm_k, k, d, Nk, (uint64_t)B * Hkv, 128) || !encode_3d(&a.tm_v, v, d, Nk, (uint64_t)B * Hkv, 128) ||
+      !encode_3d_f32(&a.tm_dq, dq, d, Nq, (uint64_t)B * Hq) || !encode_3d_f32(&a.tm_dk, dk, d, Nk, (uint64_t)B * Hkv) ||
+      !encode_3d_f32(&a.tm_dv, dv, d, Nk, (uint64_t)B * Hkv))
     return ATTN_ERR_CUDA;
   a.lse = lse;
   a.delta = static_cast<float*>(workspace);

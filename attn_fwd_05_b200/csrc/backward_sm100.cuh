@@ -34,6 +34,9 @@ struct BwdArgs {
   CUtensorMap tm_do;  // same layout as Q
   CUtensorMap tm_k;   // [B*Hkv, Nk, d] bf16, box {64, 128, 1}
   CUtensorMap tm_v;
+  CUtensorMap tm_dq;   // fp32 [B*Hq, Nq, d], box {32, 32, 1}: the gradients leave through TMA stores
+  CUtensorMap tm_dk;   // fp32 [B*Hkv, Nk, d], same boxes
+  CUtensorMap tm_dv;
   const float* lse;    // [B*Hq, Nq] natural log-sum-exp of the forward pass
   const float* delta;  // [B*Hq, Nq] rowsum(dO o O)
   float* dq;           // [B*Hq, Nq, d]
@@ -123,27 +126,46 @@ __device__ __forceinline__ void store_acc_row(uint32_t taddr, bool have, bool va
   }
 }
 
-// Columns [C0, C0 + NC) of this thread's accumulator row, as store_acc_row.
+// Columns [C0, C0 + NC) of this thread's fp32 accumulator row r (times mul), written to
+// the calling warp's rows of a staging area in the layout of TMA's 128-byte swizzled fp32
+// boxes, and stored from there with TMA: chunk i (32 columns, 128 bytes a row) of 128 rows
+// sits at stage + i * 16 KB, and row r's 16-byte granule g at g ^ (r % 8).  A warp store
+// then writes whole rows instead of touching 32 rows per instruction.  Rows at or past
+// n_rows are clipped by the tensor map; the warp stores nothing if it has none below it.
 template <int C0, int NC>
-__device__ __forceinline__ void store_acc_cols(uint32_t taddr, bool have, bool valid, float mul, float* dst) {
+__device__ __forceinline__ void store_acc_tma(uint32_t stage, int r, uint32_t taddr, bool have, float mul,
+                                              const CUtensorMap* map, int row0, int n_rows, int plane) {
+  const int lane = threadIdx.x & 31;
+  const int quad = r >> 5;
 #pragma unroll
   for (int c = C0 / 32; c < (C0 + NC) / 32; ++c) {
-    uint32_t r[32];
+    uint32_t v[32];
     if (have) {
-      tmem_ld32(taddr + c * 32, r);
-      tmem_ld_wait(r);
+      tmem_ld32(taddr + c * 32, v);
+      tmem_ld_wait(v);
     } else {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) r[i] = 0u;
+      for (int i = 0; i < 32; ++i) v[i] = 0u;
     }
-    if (valid) {
-      float4* out = reinterpret_cast<float4*>(dst + c * 32);
+    const uint32_t row = stage + (uint32_t)((c - C0 / 32) * (128 * 128) + r * 128);
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        out[i] = make_float4(__uint_as_float(r[4 * i]) * mul, __uint_as_float(r[4 * i + 1]) * mul,
-                             __uint_as_float(r[4 * i + 2]) * mul, __uint_as_float(r[4 * i + 3]) * mul);
-    }
+    for (int g = 0; g < 8; ++g)
+      st_shared_v4(row + (uint32_t)((g ^ (r & 7)) << 4), __float_as_uint(__uint_as_float(v[4 * g]) * mul),
+                   __float_as_uint(__uint_as_float(v[4 * g + 1]) * mul),
+                   __float_as_uint(__uint_as_float(v[4 * g + 2]) * mul),
+                   __float_as_uint(__uint_as_float(v[4 * g + 3]) * mul));
   }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && row0 + quad * 32 < n_rows) {
+#pragma unroll
+    for (int c = C0 / 32; c < (C0 + NC) / 32; ++c)
+      tma_store_3d(map, stage + (uint32_t)((c - C0 / 32) * (128 * 128) + quad * 32 * 128), c * 32, row0 + quad * 32,
+                   plane);
+    bulk_commit();
+    bulk_wait_all();  // the CTA exits next: the stores must have read shared memory
+  }
+  __syncwarp();
 }
 
 struct BwdBars {
@@ -399,13 +421,12 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkdv_kernel(const __grid_cons
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_final, 0, abort_flag, a.timeout_ns));
       tc_fence_after();
     }
-    if (ok) {  // half 0's warps write dK, half 1's dV
-      const bool valid = k < a.Nk;
-      const size_t row = ((size_t)bkv * a.Nk + (valid ? k : 0)) * D;
+    if (ok) {  // half 0's warps write dK, half 1's dV, each staged in one ring stage (free now)
+      const uint32_t stage = sRing + (uint32_t)(h * 2 * C::TILE_BYTES);
       if (h == 0)
-        store_acc_row<D>(tmem + lane_off + C::COL_ACC0, have, valid, a.scale, a.dk + row);
+        store_acc_tma<0, D>(stage, r, tmem + lane_off + C::COL_ACC0, have, a.scale, &a.tm_dk, k0, a.Nk, bkv);
       else
-        store_acc_row<D>(tmem + lane_off + C::COL_ACC1, have, valid, 1.0f, a.dv + row);
+        store_acc_tma<0, D>(stage, r, tmem + lane_off + C::COL_ACC1, have, 1.0f, &a.tm_dv, k0, a.Nk, bkv);
     }
   }
 
@@ -586,13 +607,12 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dq_kernel(const __grid_consta
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_final, 0, abort_flag, a.timeout_ns));
       tc_fence_after();
     }
-    if (ok) {  // each half's warps write half of the row's columns
-      const bool valid = q < a.Nq;
-      float* dst = a.dq + ((size_t)bh * a.Nq + (valid ? q : 0)) * D;
+    if (ok) {  // each half's warps write half of the row's columns, staged in the (free) ring
+      const uint32_t stage = sRing + (uint32_t)(h * (D / 64) * (128 * 128));
       if (h == 0)
-        store_acc_cols<0, D / 2>(tmem + lane_off + C::COL_ACC0, have, valid, a.scale, dst);
+        store_acc_tma<0, D / 2>(stage, r, tmem + lane_off + C::COL_ACC0, have, a.scale, &a.tm_dq, q0, a.Nq, bh);
       else
-        store_acc_cols<D / 2, D / 2>(tmem + lane_off + C::COL_ACC0, have, valid, a.scale, dst);
+        store_acc_tma<D / 2, D / 2>(stage, r, tmem + lane_off + C::COL_ACC0, have, a.scale, &a.tm_dq, q0, a.Nq, bh);
     }
   }
 
