@@ -107,7 +107,7 @@ PREFILL_PROFILES = {
 
 def profiled_traffic(profile: str, scale: float = 1.0):
     """DRAM bytes per launch from a committed ncu summary, or None when the kernel sources
-    changed since it was captured (its counters no longer describe this build)."""
+    changed since it was captured (its counters no longer describe the current kernels)."""
     path = os.path.join(ROOT, "profiles", profile)
     try:
         text = open(path).read()
