@@ -124,6 +124,43 @@ def test_fp8_bf16_store_equals_rounded_fp32_output(B, Hq, Hkv, Nq, Nk, causal, c
     assert np.array_equal(l16, l32)
 
 
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["gqa_causal_2k", "gqa_causal_16k"])
+def test_fp8_full_size_sampled(name, cuda_device):
+    # the FP8 bench's launch on the whole workload (quantized on the GPU, bf16 O); sampled
+    # rows against the exact attention of the dequantized inputs, within the bound above
+    # plus half a bf16 unit for the output's own rounding
+    s = synth.WORKLOADS[name]
+    q, k, v = synth.prefill_inputs(s, synth.workload_seed(name))
+    dev = torch.device("cuda:0")
+    q8, qs = ab.attn_quantize_fp8(q.to(dev), 128)
+    k8, ks = ab.attn_quantize_fp8(k.to(dev), 128)
+    v8, vs = ab.attn_quantize_fp8(v.to(dev), s.Nk)
+    del q, k, v
+    o = torch.empty((s.B, s.Hq, s.Nq, s.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((s.B, s.Hq, s.Nq), dtype=torch.float32, device=dev)
+    scale = synth.default_scale(s.d)
+    ab.attn_fwd_fp8(q8, qs, k8, ks, v8, vs[..., 0].contiguous(), o, lse, s.causal, scale)
+    assert ab.attn_get_device_status() == 0
+    rng = np.random.default_rng(41)
+    for trial in range(4):
+        b, h = int(rng.integers(s.B)), int(rng.integers(s.Hq))
+        kv = kv_head_of(h, s.Hq, s.Hkv)
+        rows = np.sort(rng.choice(s.Nq, 6, replace=False))
+        rows[0] = 0 if trial == 0 else rows[0]
+        rows[-1] = s.Nq - 1 if trial == 1 else rows[-1]
+        qd = dequantize(q8[b, h].cpu().numpy(), qs[b, h].cpu().numpy())[rows]
+        kd = dequantize(k8[b, kv].cpu().numpy(), ks[b, kv].cpu().numpy())
+        vd = dequantize(v8[b, kv].cpu().numpy(), vs[b, kv].cpu().numpy(), block=s.Nk)
+        ref_o, ref_l, P = attention_head(qd, kd, vd, scale, s.causal, rows=rows, nq=s.Nq, want_p=True)
+        got = o[b, h, torch.from_numpy(rows).to(dev)].double().cpu().numpy()
+        bound = (2.0 ** -4 * P + 2.0 ** -18 * (P > 0)) @ np.abs(vd) + 1e-5 + np.abs(got) * 2.0 ** -9
+        err = np.abs(got - ref_o)
+        assert np.all(err <= bound), f"{name} head {b},{h}: max excess {(err - bound).max():.3e}"
+        gl = lse[b, h, torch.from_numpy(rows).to(dev)].double().cpu().numpy()
+        assert np.all(np.abs(gl - ref_l) <= 1e-3)
+
+
 def test_fp8_rejects_other_head_dims(cuda_device):
     dev = torch.device("cuda:0")
     x = torch.zeros((1, 1, 16, 64), dtype=torch.uint8, device=dev)
