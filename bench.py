@@ -78,6 +78,8 @@ PROFILE_SOURCES = {
     "attn_decode_split_paged_decode.md": ("attn_api.cu", "decode_sm100.cuh", "sm100_common.cuh"),
     "attn_bwd_gqa_causal_2k.md": ("attn_api.cu", "backward_sm100.cuh", "sm100_common.cuh"),
     "attn_fwd_fp8_gqa_causal_2k.md": ("attn_api.cu", "fwd_fp8_sm100.cuh", "sm100_common.cuh"),
+    "attn_fwd_fp8_gqa_causal_16k.md": ("attn_api.cu", "fwd_fp8_sm100.cuh", "sm100_common.cuh"),
+    "attn_bwd_gqa_causal_16k.md": ("attn_api.cu", "backward_sm100.cuh", "sm100_common.cuh"),
 }
 
 
@@ -476,7 +478,8 @@ def run_backward(args, dist):
                    "parallelism": f"independent replicas x{dist.world} (no data-path collective)"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_tflops"],
-                     "traffic": profiled_traffic("attn_bwd_gqa_causal_2k.md") if name == "gqa_causal_2k" else None,
+                     "traffic": profiled_traffic(f"attn_bwd_{name}.md") if name in ("gqa_causal_2k", "gqa_causal_16k")
+                     else None,
                      "peak_source": f"{peak_src} bf16_tflops (burst cuBLAS)",
                      "kernel": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel + attn_bwd_delta_kernel (one call)",
                      "flops_per_launch": flops, "median_ms": statistics.median(ms)},
@@ -586,8 +589,8 @@ def run_fp8(args, dist):
                    "parallelism": f"independent replicas x{dist.world} (no data-path collective)"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak,
-                     "traffic": profiled_traffic("attn_fwd_fp8_gqa_causal_2k.md")
-                     if args.workload == "gqa_causal_2k_fp8" else None,
+                     "traffic": profiled_traffic(f"attn_fwd_fp8_{args.workload[:-len('_fp8')]}.md")
+                     if args.workload in ("gqa_causal_2k_fp8", "gqa_causal_16k_fp8") else None,
                      "peak_source": f"2 x {peak_src} bf16_tflops (nominal e4m3 : bf16 dense ratio)",
                      "kernel": "attn_fwd_fp8_kernel", "flops_per_launch": flops, "median_ms": statistics.median(ms)},
         "gpu_launches": K, "clocks": clk,
