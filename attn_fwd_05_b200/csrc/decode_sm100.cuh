@@ -56,57 +56,100 @@ struct DecArgs {
 
 // ------------------------------------------------------------------ plan
 
-// chunk_prefix[s] = number of work chunks of sequences < s, and item_map[k] describes
-// flat chunk k (one CTA, any S).  With the map a work item's sequence is one load, not
-// a search: dependent loads are slow while the split pass saturates HBM.
+// chunk_prefix[s] = number of work chunks of sequences < s (the merge finds a sequence's
+// partials by chunk index), and item_map[k] describes work chunk k (one CTA, any S).  With
+// the map a work item's sequence is one load, not a search: dependent loads are slow while
+// the split pass saturates HBM.
+//
+// The chunks are listed longest first, because the split kernel hands them out round-robin:
+// every full chunk (kDecChunkTok tokens) in sequence order, then each sequence's shorter
+// last chunk, longest first (ties by sequence; in sequence order beyond kPlanSortMax
+// sequences), so that the last rounds get the short chunks.
+constexpr int kPlanSortMax = 2048;
+
+// Block-wide exclusive scan (every thread of the block calls it with its value): returns
+// *carry plus the sum of the values of the lower threads, and adds the block's total to
+// *carry.  warp_sums: 32 ints of shared memory.
+__device__ __forceinline__ int plan_scan(int v, int* carry, int* warp_sums) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (int)(blockDim.x >> 5);
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int t = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    warp_sums[lane] = t;  // inclusive scan of the warp totals
+  }
+  __syncthreads();
+  const int before = *carry + (w > 0 ? warp_sums[w - 1] : 0) + (x - v);
+  __syncthreads();
+  if (threadIdx.x == 0) *carry += warp_sums[nw - 1];
+  __syncthreads();
+  return before;
+}
+
 __global__ void attn_decode_plan_kernel(const int32_t* __restrict__ seq_lens, int S, int max_tokens,
                                         int* __restrict__ chunk_prefix, int4* __restrict__ item_map) {
-  __shared__ int carry;
+  __shared__ int carry_all, carry_full, carry_part;
   __shared__ int warp_sums[32];
-  if (threadIdx.x == 0) carry = 0;
+  __shared__ int tail_len[kPlanSortMax];  // tokens in each sequence's last, shorter chunk (0: none)
+  if (threadIdx.x == 0) carry_all = carry_full = carry_part = 0;
   __syncthreads();
+  // pass 1: the prefix of all chunks, and the full chunks in sequence order
   for (int base = 0; base < S; base += blockDim.x) {
     const int s = base + threadIdx.x;
-    int n = 0;
+    int len = 0;
     if (s < S) {
-      int len = seq_lens[s];
+      len = seq_lens[s];
       if (len < 0 || len > max_tokens) {
         latch_status(ATTN_ERR_INVALID_ARG);
         len = 0;
       }
-      n = (len + kDecChunkTok - 1) / kDecChunkTok;
     }
-    // block-wide exclusive scan
-    int x = n;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) warp_sums[w] = x;
-    __syncthreads();
-    if (w == 0) {
-      int v = lane < (int)(blockDim.x >> 5) ? warp_sums[lane] : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += y;
-      }
-      warp_sums[lane] = v;  // inclusive scan of warp totals
-    }
-    __syncthreads();
-    const int before = carry + (w > 0 ? warp_sums[w - 1] : 0) + (x - n);
+    const int n_full = len / kDecChunkTok;
+    const int tail = len % kDecChunkTok;
+    const int before_all = plan_scan(n_full + (tail != 0 ? 1 : 0), &carry_all, warp_sums);
+    const int before_full = plan_scan(n_full, &carry_full, warp_sums);
     if (s < S) {
-      chunk_prefix[s] = before;
-      const int len = n > 0 ? seq_lens[s] : 0;
-      for (int c = 0; c < n; ++c) item_map[before + c] = make_int4(s, c, len, 0);
+      chunk_prefix[s] = before_all;
+      for (int c = 0; c < n_full; ++c) item_map[before_full + c] = make_int4(s, c, len, 0);
+      if (S <= kPlanSortMax) tail_len[s] = tail;
     }
-    __syncthreads();
-    if (threadIdx.x == 0) carry += warp_sums[(blockDim.x >> 5) - 1];
-    __syncthreads();
   }
-  if (threadIdx.x == 0) chunk_prefix[S] = carry;
+  __syncthreads();
+  const int total_full = carry_full;
+  if (threadIdx.x == 0) chunk_prefix[S] = carry_all;
+  // pass 2: the shorter last chunks after the full ones
+  for (int base = 0; base < S; base += blockDim.x) {
+    const int s = base + threadIdx.x;
+    int len = 0;
+    if (s < S) {
+      len = seq_lens[s];
+      if (len < 0 || len > max_tokens) len = 0;
+    }
+    const int tail = len % kDecChunkTok;
+    int slot;
+    if (S <= kPlanSortMax) {  // rank by (length descending, sequence)
+      slot = 0;
+      if (tail != 0)
+        for (int t = 0; t < S; ++t) {
+          const int o = tail_len[t];
+          slot += (o > tail || (o == tail && t < s)) ? 1 : 0;
+        }
+    } else {
+      slot = plan_scan(tail != 0 ? 1 : 0, &carry_part, warp_sums);
+    }
+    if (s < S && tail != 0) item_map[total_full + slot] = make_int4(s, len / kDecChunkTok, len, 0);
+  }
 }
 
 // ------------------------------------------------------------------ split kernel
