@@ -61,6 +61,21 @@ def test_decode_matches_oracle(lens, Hq, Hkv, d, ps, cuda_device):
     compare_lse(lse, ref_l)
 
 
+def test_more_sequences_than_the_plan_sorts(cuda_device):
+    # beyond 2048 sequences the plan keeps the shorter last chunks in sequence order
+    rng = np.random.default_rng(77)
+    lens = [int(x) for x in rng.integers(0, 200, 2100)]
+    for i in range(0, 2100, 50):  # some sequences with a full 2048-token chunk, one exactly
+        lens[i] = 2048 + (0 if i == 0 else int(rng.integers(1, 400)))
+    kv = make(lens, Hq=4, Hkv=1, d=64, page_size=16, seed=78)
+    scale = 1.0 / math.sqrt(64)
+    ref_o, ref_l = decode_paged(kv.q, kv.k_pool, kv.v_pool, kv.block_table, kv.seq_lens, 16, scale)
+    o, lse, status = run_decode(kv, scale)
+    assert status == 0, ab.attn_status_string(status)
+    compare_o(o, ref_o, bf16_out=True)
+    compare_lse(lse, ref_l)
+
+
 def test_zero_length_sequence(cuda_device):
     kv = make([0, 40, 0], Hq=4, Hkv=2)
     o, lse, status = run_decode(kv, 0.1)
