@@ -45,6 +45,10 @@ SIGNATURES = {
     "attn_decode_paged_noalloc_max_scratch": (ctypes.c_size_t, []),
     "attn_debug_watchdog": (_I, [ctypes.c_uint64, _P]),
     "attn_debug_exp2": (_I, [_P, _P, _I, _P]),
+    "attn_debug_fwd_stall": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _I, _I,
+                                  ctypes.c_uint64, _P]),
+    "attn_debug_decode_stall": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P,
+                                     ctypes.c_size_t, _I, _I, ctypes.c_uint64, _P]),
     "attn_get_device_status": (_I, [_P]),
     "attn_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -291,6 +295,40 @@ def attn_get_device_status(stream=None) -> int:
 
 def attn_debug_watchdog(timeout_ns: int, stream=None) -> None:
     _check(load_library().attn_debug_watchdog(int(timeout_ns), _stream(stream)), "attn_debug_watchdog")
+
+
+def attn_debug_fwd_stall(q, k, v, o, lse, causal: bool, scale: float, stall_cta: int, stall_fill: int,
+                         timeout_ns: int, stream=None) -> None:
+    """attn_fwd_ex with one K/V ring fill left out in one CTA and pipeline waits limited to
+    timeout_ns: exercises the kernel's timeout wind-down (testing only)."""
+    lib = load_library()
+    ptrs, dims = _fwd_shapes(q, k, v, o, lse)
+    st = lib.attn_debug_fwd_stall(*ptrs, *dims, float(scale), int(bool(causal)), int(stall_cta), int(stall_fill),
+                                  int(timeout_ns), _stream(stream))
+    _check(st, "attn_debug_fwd_stall")
+
+
+def attn_debug_decode_stall(q, k_pool, v_pool, block_table, seq_lens, page_size: int, o, lse, scale: float,
+                            workspace: torch.Tensor, stall_cta: int, stall_piece: int, timeout_ns: int,
+                            stream=None) -> None:
+    """attn_decode_paged with one K/V piece left out in one CTA of the split kernel and
+    pipeline waits limited to timeout_ns (testing only)."""
+    lib = load_library()
+    S, Hq, d = q.shape
+    num_pages, Hkv, ps, d2 = k_pool.shape
+    if ps != page_size or d2 != d or tuple(v_pool.shape) != tuple(k_pool.shape):
+        raise ValueError("pools must be [num_pages, Hkv, page_size, d]")
+    if block_table.dim() != 2 or block_table.shape[0] != S:
+        raise ValueError("block_table must be [num_seqs, max_pages_per_seq]")
+    st = lib.attn_debug_decode_stall(
+        _dev(q, "q", torch.bfloat16, 3), _dev(k_pool, "k_pool", torch.bfloat16, 4),
+        _dev(v_pool, "v_pool", torch.bfloat16, 4), _dev(block_table, "block_table", torch.int32, 2),
+        _dev(seq_lens, "seq_lens", torch.int32, 1), page_size, _dev(o, "o", torch.bfloat16, 3),
+        None if lse is None else _dev(lse, "lse", torch.float32, 2), S, Hq, Hkv, d, num_pages,
+        block_table.shape[1], float(scale), _dev(workspace, "workspace", workspace.dtype),
+        workspace.numel() * workspace.element_size(), int(stall_cta), int(stall_piece), int(timeout_ns),
+        _stream(stream))
+    _check(st, "attn_debug_decode_stall")
 
 
 def attn_debug_exp2(x: torch.Tensor, y: torch.Tensor, stream=None) -> None:

@@ -276,7 +276,9 @@ constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB
 static __device__ __align__(256) uint8_t g_decode_scratch[kStaticScratchBytes];
 
 // Device address of g_decode_scratch on the current device (looked up on the first
-// call for that device), or nullptr if the lookup failed.
+// call for that device), or nullptr if the lookup failed.  The address is valid for the
+// primary context it was looked up in: a device reset invalidates it for the rest of the
+// process.
 void* static_scratch_address() {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
@@ -317,9 +319,15 @@ const char* attn_status_string(int s) {
 
 namespace {
 
+// Failure-path testing: which ring fill of which CTA to leave out, and the wait limit.
+struct DebugStall {
+  int cta, fill;
+  uint64_t timeout_ns;
+};
+
 attn_status fwd_common(const void* q, const void* k, const void* v, void* o, int o_dtype, float* lse, int B, int Hq,
                        int Hkv, int Nq, int Nk, int d, float scale, int causal, int window, const uint8_t* block_mask,
-                       void* stream) {
+                       void* stream, const DebugStall* dbg = nullptr) {
   if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
   if (window < 0 || (window > 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
@@ -371,7 +379,9 @@ attn_status fwd_common(const void* q, const void* k, const void* v, void* o, int
   a.scale_log2 = scale * 1.4426950408889634f;
   a.pair_heads = (a.group % 2 == 0) ? 1 : 0;
   a.n_qtiles = (Nq + 127) / 128;
-  a.timeout_ns = kDefaultTimeoutNs;
+  a.timeout_ns = dbg != nullptr ? dbg->timeout_ns : kDefaultTimeoutNs;
+  a.dbg_stall_cta = dbg != nullptr ? dbg->cta : -1;
+  a.dbg_stall_fill = dbg != nullptr ? dbg->fill : -1;
   // a window wider than every row's visible prefix hides nothing
   a.window = ((long long)window >= (long long)Nk + 1 || window == 0) ? 0 : window;
   a.block_mask = block_mask;
@@ -550,16 +560,27 @@ size_t attn_decode_paged_workspace_size(int num_seqs, int Hq, int Hkv, int d, in
   return L.total;
 }
 
-attn_status attn_decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_table,
-                              const int32_t* seq_lens, int page_size, void* o, float* lse, int num_seqs, int Hq,
-                              int Hkv, int d, int num_pages, int max_pages_per_seq, float scale, void* workspace,
-                              size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Checks of a decode call's arguments, made on the host before anything touches the
+// device.  ATTN_OK with *empty set: no sequence, nothing to launch.  On ATTN_OK, *L is
+// the workspace layout.
+attn_status decode_check(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_table,
+                         const int32_t* seq_lens, int page_size, const void* o, const float* lse, int num_seqs,
+                         int Hq, int Hkv, int d, int num_pages, int max_pages_per_seq, float scale, bool* empty,
+                         DecodeLayout* L) {
+  *empty = false;
   if (num_seqs < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || num_pages < 0 || max_pages_per_seq <= 0)
     return ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.0f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
   if (page_size != 16 && page_size != 32 && page_size != 64) return ATTN_ERR_UNSUPPORTED;
-  if (num_seqs == 0) return ATTN_OK;
+  if (num_seqs == 0) {
+    *empty = true;
+    return ATTN_OK;
+  }
   if (q == nullptr || o == nullptr || block_table == nullptr || seq_lens == nullptr) return ATTN_ERR_INVALID_ARG;
   if (num_pages > 0 && (k_pool == nullptr || v_pool == nullptr)) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 4) || !aligned(o, 4) || !aligned(block_table, 4) || !aligned(seq_lens, 4) ||
@@ -567,8 +588,19 @@ attn_status attn_decode_paged(const void* q, const void* k_pool, const void* v_p
     return ATTN_ERR_ALIGNMENT;
   if ((long long)num_pages * Hkv > 0x7fffffffLL || (long long)num_seqs * Hq > 0x7fffffffLL)
     return ATTN_ERR_INVALID_ARG;
+  if (!decode_layout(num_seqs, Hq, d, max_pages_per_seq, page_size, L)) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+attn_status decode_common(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_table,
+                          const int32_t* seq_lens, int page_size, void* o, float* lse, int num_seqs, int Hq, int Hkv,
+                          int d, int num_pages, int max_pages_per_seq, float scale, void* workspace,
+                          size_t workspace_bytes, void* stream, const DebugStall* dbg) {
   DecodeLayout L;
-  if (!decode_layout(num_seqs, Hq, d, max_pages_per_seq, page_size, &L)) return ATTN_ERR_INVALID_ARG;
+  bool empty = false;
+  const attn_status chk = decode_check(q, k_pool, v_pool, block_table, seq_lens, page_size, o, lse, num_seqs, Hq, Hkv,
+                                       d, num_pages, max_pages_per_seq, scale, &empty, &L);
+  if (chk != ATTN_OK || empty) return chk;
   if (workspace == nullptr || workspace_bytes < L.total) return ATTN_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return ATTN_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -604,7 +636,9 @@ attn_status attn_decode_paged(const void* q, const void* k_pool, const void* v_p
   a.max_pages = max_pages_per_seq;
   a.max_chunks = L.max_chunks;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.timeout_ns = kDefaultTimeoutNs;
+  a.timeout_ns = dbg != nullptr ? dbg->timeout_ns : kDefaultTimeoutNs;
+  a.dbg_stall_cta = dbg != nullptr ? dbg->cta : -1;
+  a.dbg_stall_piece = dbg != nullptr ? dbg->fill : -1;
   const long long max_items = (long long)num_seqs * L.max_chunks * Hkv * a.n_hgroups;
   if (max_items > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
   switch (d) {
@@ -614,23 +648,34 @@ attn_status attn_decode_paged(const void* q, const void* k_pool, const void* v_p
   }
 }
 
+}  // namespace
+
+extern "C" {
+
+attn_status attn_decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_table,
+                              const int32_t* seq_lens, int page_size, void* o, float* lse, int num_seqs, int Hq,
+                              int Hkv, int d, int num_pages, int max_pages_per_seq, float scale, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  return decode_common(q, k_pool, v_pool, block_table, seq_lens, page_size, o, lse, num_seqs, Hq, Hkv, d, num_pages,
+                       max_pages_per_seq, scale, workspace, workspace_bytes, stream, nullptr);
+}
+
 attn_status attn_decode_paged_noalloc(const void* q, const void* k_pool, const void* v_pool,
                                       const int32_t* block_table, const int32_t* seq_lens, int page_size, void* o,
                                       float* lse, int num_seqs, int Hq, int Hkv, int d, int num_pages,
                                       int max_pages_per_seq, float scale, void* stream) {
-  // Same checks as attn_decode_paged, so that a rejected call never touches the device.
-  if (num_seqs < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || num_pages < 0 || max_pages_per_seq <= 0)
-    return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
-  if (page_size != 16 && page_size != 32 && page_size != 64) return ATTN_ERR_UNSUPPORTED;
-  if (num_seqs == 0) return ATTN_OK;
-  const size_t need = attn_decode_paged_workspace_size(num_seqs, Hq, Hkv, d, max_pages_per_seq, page_size);
-  if (need == 0) return ATTN_ERR_INVALID_ARG;
-  if (need > kStaticScratchBytes) return ATTN_ERR_TOO_LARGE;
+  // Every argument check of attn_decode_paged comes first, so that a rejected call never
+  // touches the device (not even the symbol lookup of the first call).
+  DecodeLayout L;
+  bool empty = false;
+  const attn_status chk = decode_check(q, k_pool, v_pool, block_table, seq_lens, page_size, o, lse, num_seqs, Hq, Hkv,
+                                       d, num_pages, max_pages_per_seq, scale, &empty, &L);
+  if (chk != ATTN_OK || empty) return chk;
+  if (L.total > kStaticScratchBytes) return ATTN_ERR_TOO_LARGE;
   void* scratch = static_scratch_address();
   if (scratch == nullptr) return ATTN_ERR_CUDA;
-  return attn_decode_paged(q, k_pool, v_pool, block_table, seq_lens, page_size, o, lse, num_seqs, Hq, Hkv, d,
-                           num_pages, max_pages_per_seq, scale, scratch, kStaticScratchBytes, stream);
+  return decode_common(q, k_pool, v_pool, block_table, seq_lens, page_size, o, lse, num_seqs, Hq, Hkv, d, num_pages,
+                       max_pages_per_seq, scale, scratch, kStaticScratchBytes, stream, nullptr);
 }
 
 size_t attn_decode_paged_noalloc_max_scratch(void) { return kStaticScratchBytes; }
@@ -639,6 +684,26 @@ attn_status attn_debug_watchdog(uint64_t timeout_ns, void* stream) {
   if (timeout_ns == 0 || timeout_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;
   attn::attn_watchdog_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
   return launch_status();
+}
+
+attn_status attn_debug_fwd_stall(const void* q, const void* k, const void* v, void* o, int o_dtype, float* lse, int B,
+                                 int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, int stall_cta,
+                                 int stall_fill, uint64_t timeout_ns, void* stream) {
+  if (d > 128) return ATTN_ERR_UNSUPPORTED;  // the two-tile kernel's producer carries the switch
+  if (stall_cta < 0 || stall_fill < 0 || timeout_ns == 0 || timeout_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;
+  const DebugStall dbg{stall_cta, stall_fill, timeout_ns};
+  return fwd_common(q, k, v, o, o_dtype, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, nullptr, stream, &dbg);
+}
+
+attn_status attn_debug_decode_stall(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_table,
+                                    const int32_t* seq_lens, int page_size, void* o, float* lse, int num_seqs, int Hq,
+                                    int Hkv, int d, int num_pages, int max_pages_per_seq, float scale, void* workspace,
+                                    size_t workspace_bytes, int stall_cta, int stall_piece, uint64_t timeout_ns,
+                                    void* stream) {
+  if (stall_cta < 0 || stall_piece < 0 || timeout_ns == 0 || timeout_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;
+  const DebugStall dbg{stall_cta, stall_piece, timeout_ns};
+  return decode_common(q, k_pool, v_pool, block_table, seq_lens, page_size, o, lse, num_seqs, Hq, Hkv, d, num_pages,
+                       max_pages_per_seq, scale, workspace, workspace_bytes, stream, &dbg);
 }
 
 attn_status attn_debug_exp2(const float* x, float* y, int n, void* stream) {

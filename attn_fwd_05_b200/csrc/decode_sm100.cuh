@@ -52,6 +52,10 @@ struct DecArgs {
   int S, Hq, Hkv, group, n_hgroups, page_size, num_pages, max_pages, max_chunks;
   float scale_log2;
   uint64_t timeout_ns;
+  // failure-path testing only (-1 in every normal call): CTA dbg_stall_cta leaves its
+  // piece number dbg_stall_piece out, so the wait for it runs out after timeout_ns
+  int dbg_stall_cta;
+  int dbg_stall_piece;
 };
 
 // ------------------------------------------------------------------ plan
@@ -259,9 +263,10 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
           const int pg = __shfl_sync(0xffffffffu, pages, i);
           const int st = gp % C::NST;
           const int use = gp / C::NST;
+          const bool stall = a.dbg_stall_cta == (int)blockIdx.x && gp == a.dbg_stall_piece;
           if (lane == 0) {
             if (use > 0 && !mbar_wait(&misc->empty[st], (use - 1) & 1, abort_flag, a.timeout_ns)) ok = false;
-            if (ok) {
+            if (ok && !stall) {
               const bool good = pg >= 0 && pg < a.num_pages;
               misc->stage_ok[st] = good ? 1 : 0;
               if (good) {
@@ -300,6 +305,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
     if (lane == 0) {  // drain copies still in flight
       for (int st = 0; st < C::NST && st < gp; ++st) {
         const int last_use = (gp - 1 - st) / C::NST;
+        if (a.dbg_stall_cta == (int)blockIdx.x && st + last_use * C::NST == a.dbg_stall_piece) continue;
         mbar_wait(&misc->full[st], last_use & 1, abort_flag, a.timeout_ns, false);
       }
     }

@@ -61,7 +61,16 @@ struct FwdArgs {
   int window;
   const uint8_t* block_mask;
   int nkt;  // ceil(Nk / 128)
+  // failure-path testing only (-1 in every normal call): CTA dbg_stall_cta leaves its K/V
+  // ring fill number dbg_stall_fill out, so the wait for it runs out after timeout_ns
+  int dbg_stall_cta;
+  int dbg_stall_fill;
 };
+
+// Is ring fill `fill` of this CTA the one a failure-path test leaves out?
+__device__ __forceinline__ bool stalled_fill(int stall_cta, int stall_fill, int fill) {
+  return stall_cta == (int)blockIdx.x && fill == stall_fill;
+}
 
 constexpr int kMaskBlock = 128;  // block size of the block-sparse map
 constexpr int kMaxVisits = 2048;  // blocks a CTA may visit under a block-sparse map
@@ -576,6 +585,10 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
         const int st = seq % C::NSTAGE;
         const int use = seq / C::NSTAGE;
         if (use > 0 && !mbar_wait(&bars->kv_empty[st], (use - 1) & 1, abort_flag, a.timeout_ns)) return false;
+        if (stalled_fill(a.dbg_stall_cta, a.dbg_stall_fill, seq)) {  // never armed, never completes
+          ++seq;
+          return true;
+        }
         mbar_arrive_expect_tx(&bars->kv_full[st], C::KV_BYTES);
         const CUtensorMap* map = kv ? &a.tm_v : &a.tm_k;
 #pragma unroll
@@ -618,6 +631,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
         if (nql[t] > 0) mbar_wait(&bars->q_full[t], (nql[t] - 1) & 1, abort_flag, a.timeout_ns, false);
       for (int st = 0; st < C::NSTAGE && st < seq; ++st) {
         const int last_use = (seq - 1 - st) / C::NSTAGE;  // index of the last fill of stage st
+        if (stalled_fill(a.dbg_stall_cta, a.dbg_stall_fill, st + last_use * C::NSTAGE)) continue;
         mbar_wait(&bars->kv_full[st], last_use & 1, abort_flag, a.timeout_ns, false);
       }
     }

@@ -11,9 +11,13 @@ prefill launch starts with a cold L2 for its own inputs.
 
 Printed (rank 0, one JSON line): prefill TFLOP/s as `value` (causal FLOPs counted as
 half of 4*B*Hq*Nq*Nk*d), the decode KV-read GB/s in `decode`, roofline fractions
-against MEASURED_PEAKS.json, the end-to-end figure through the public API with host
-buffers (`e2e`), the fp64 CPU oracle timed on a bounded sample (`cpu_baseline`), and
-the SM clocks sampled during the run.
+against MEASURED_PEAKS.json, the end-to-end figures through the public API with host
+buffers (`e2e` for the prefill, `decode.e2e` for the decode), the fp64 CPU oracle timed
+on a bounded sample (`cpu_baseline`), and the SM clocks sampled during the run.  After
+the timed step, the other prefill configurations (the tiny d=64 case, the 16K
+long-context case and the peaked d=256 case) are each timed on their own, L2 flushed
+before every launch, and reported under `workloads` with their own roofline, clocks
+and CPU baseline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload serving_step|gqa_causal_16k|peaked_mha_d256|tiny_mha_d64]
@@ -62,6 +66,8 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="bounded CPU-baseline sample length")
     p.add_argument("--decode-seqs", type=int, default=64,
                    help="sequences in the decode batch (64 is the workload; fewer only for small profiles)")
+    p.add_argument("--no-other-workloads", action="store_true",
+                   help="serving step only: skip the per-workload records of the other prefill configs")
     return p.parse_args()
 
 
@@ -293,8 +299,16 @@ def oracle_prefill_sample(shape, q, k, v, seconds: float, max_heads=None):
             break
     dt = time.perf_counter() - t0
     flops = counts.prefill_flops(1, done, shape.Nq, shape.Nk, shape.d, shape.causal)
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"{done} of {len(heads)} (batch, head) pairs of the workload, {dt:.1f} s, fp64 numpy"}
+    full = counts.prefill_flops(shape.B, shape.Hq, shape.Nq, shape.Nk, shape.d, shape.causal)
+    rate = flops / dt
+    rec = {"value": rate / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+           "sample": f"{done} of {len(heads)} (batch, head) pairs of the workload, {dt:.1f} s, fp64 numpy"}
+    if done < len(heads):
+        rec["workload_s_extrapolated"] = full / rate
+        rec["sample"] += "; the whole workload's time is extrapolated linearly from the sample's rate"
+    else:
+        rec["workload_s"] = dt
+    return rec
 
 
 def oracle_decode_sample(dec, seconds: float):
@@ -722,14 +736,133 @@ def run_ours(args, dist):
 
     if not args.no_e2e:
         line["e2e"] = e2e_prefill(args, ab, pre, shape, scale, flops, dev, stream, dist)
+        if dec is not None:
+            line["decode"]["e2e"] = e2e_decode(args, ab, dec, scale, dev, stream, dist)
     if dist.rank == 0 and N == 1 and not args.no_cpu_baseline:
         q, k, v = pre["host"]
         line["cpu_baseline"] = oracle_prefill_sample(shape, q, k, v, args.cpu_seconds)
         if dec is not None:
             line["decode"]["cpu_baseline"] = oracle_decode_sample(dec, max(2.0, args.cpu_seconds / 3))
+    if args.workload == "serving_step" and not args.no_other_workloads:
+        # the other prefill configurations, each timed on its own (not part of the step)
+        del pre, dec
+        torch.cuda.empty_cache()
+        line["workloads"] = {name: prefill_record(args, ab, name, dev, stream, dist, peaks, peak_src)
+                             for name in OTHER_PREFILL}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+OTHER_PREFILL = ("tiny_mha_d64", "gqa_causal_16k", "peaked_mha_d256")
+
+
+def prefill_record(args, ab, name, dev, stream, dist, peaks, peak_src):
+    """One prefill workload timed on its own: W warm-up launches, then K launches, each
+    after a 256 MB write that flushes L2, timed by CUDA events on the launching stream.
+    Returns the workload's record (median and mean launch time, TFLOP/s, roofline against
+    the measured peak, DRAM traffic from the committed ncu summary, clocks, and on rank 0
+    at N = 1 the oracle's rate on a bounded sample)."""
+    shape = synth.WORKLOADS[name]
+    seed = rank_seed(synth.workload_seed(name), dist.rank)
+    pre = make_prefill(shape, seed, dev)
+    qd, kd, vd = pre["dev"]
+    scale = synth.default_scale(shape.d)
+    flops = counts.prefill_flops(shape.B, shape.Hq, shape.Nq, shape.Nk, shape.d, shape.causal)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    K = max(3, min(args.steps, 100 if flops < 1e12 else 30))
+
+    def launch():
+        ab.attn_fwd(qd, kd, vd, pre["o"], pre["lse"], shape.causal, scale, stream)
+
+    clocks = ClockSampler(dist.local)
+    clocks.start()
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        launch()
+    torch.cuda.synchronize(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K)]
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        flush.zero_()
+        ev[2 * i].record(stream)
+        launch()
+        ev[2 * i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clk = clocks.stop()
+    st = ab.attn_get_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"kernel fault in the timed region of {name}: {ab.attn_status_string(st)}")
+    ms = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K)]
+    tot = dist.max(sum(ms))
+    achieved = flops / (sum(ms) / K * 1e-3) / 1e12
+    kname = "attn_fwd_pingpong_kernel<%d>" % shape.d if shape.d <= 128 else "attn_fwd_single_kernel<256>"
+    rec = {
+        "metric": "attn fwd TFLOPS & % of BF16 tensor peak", "unit": "TFLOP/s",
+        "value": dist.world * flops * K / (tot * 1e-3) / 1e12, "steps": K, "ms_per_launch": tot / K,
+        "median_ms": statistics.median(ms),
+        "shape": {"B": shape.B, "Hq": shape.Hq, "Hkv": shape.Hkv, "Nq": shape.Nq, "Nk": shape.Nk, "d": shape.d,
+                  "causal": shape.causal, "qk_std": shape.qk_std},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": profiled_traffic(PREFILL_PROFILES[name]) if name in PREFILL_PROFILES else None,
+                     "peak_source": f"{peak_src} bf16_tflops (burst cuBLAS); frac of the sustained figure "
+                                    f"{achieved / peaks['bf16_tflops_sustained']:.3f}",
+                     "kernel": kname, "flops_per_launch": flops},
+        "l2": "L2 flushed before every launch by writing a 256 MB buffer",
+        "clocks": clk, "gpu_launches": K,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        q, k, v = pre["host"]
+        rec["cpu_baseline"] = oracle_prefill_sample(shape, q, k, v, args.cpu_seconds)
+    return rec
+
+
+def e2e_decode(args, ab, dec, scale, dev, stream, dist):
+    """The decode metric through the public API with host buffers: every step copies the
+    step's inputs (the query tokens, the block table and the sequence lengths) from
+    pinned host memory, runs attn_decode_paged, and copies O and LSE back, all inside the
+    timed region.  The paged K/V pools are the cache: they stay resident in HBM across
+    steps, as a serving engine keeps them."""
+    qh = dec["kv"].q.pin_memory()
+    th = dec["kv"].block_table.pin_memory()
+    lh = dec["kv"].seq_lens.pin_memory()
+    oh = torch.empty(dec["o"].shape, dtype=torch.bfloat16).pin_memory()
+    lseh = torch.empty(dec["lse"].shape, dtype=torch.float32).pin_memory()
+    qd = torch.empty_like(qh, device=dev)
+    td = torch.empty_like(th, device=dev)
+    ld = torch.empty_like(lh, device=dev)
+
+    def step():
+        qd.copy_(qh, non_blocking=True)
+        td.copy_(th, non_blocking=True)
+        ld.copy_(lh, non_blocking=True)
+        ab.attn_decode_paged(qd, dec["k_pool"], dec["v_pool"], td, ld, dec["shape"].page_size, dec["o"], dec["lse"],
+                             scale, dec["ws"], stream)
+        oh.copy_(dec["o"], non_blocking=True)
+        lseh.copy_(dec["lse"], non_blocking=True)
+
+    K = max(3, min(args.steps, 20))
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    a.record(stream)
+    for _ in range(K):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = dist.max(a.elapsed_time(b))
+    h2d = sum(t.numel() * t.element_size() for t in (qh, th, lh))
+    d2h = oh.numel() * 2 + lseh.numel() * 4
+    return {"value": dist.world * dec["kv_bytes"] * K / (ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": K,
+            "note": "paged K/V pools resident in HBM (the cache); query, block table and lengths copied in, "
+                    "O and LSE copied out every step"}
 
 
 def e2e_prefill(args, ab, pre, shape, scale, flops, dev, stream, dist):

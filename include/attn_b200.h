@@ -267,7 +267,11 @@ attn_status attn_decode_paged(const void* q, const void* k_pool, const void* v_p
  *   page_size) exceeds that size; other argument errors are those of attn_decode_paged.
  *   The first call on a device looks up the device address of the static array (a
  *   cudaGetSymbolAddress on the current device); make that first call before any
- *   stream capture.
+ *   stream capture.  The address is kept for the life of the process: after a
+ *   cudaDeviceReset, or anything else that destroys the device's primary context, this
+ *   entry point must not be called again in the same process (it would pass the old
+ *   address to the kernels).  All argument checks run before that lookup, so a call
+ *   rejected for its arguments touches no device.
  *   Every call shares the one array and leaves its contents behind; nothing in it has
  *   to start at zero (each call rewrites what it later reads).  Calls that overlap on
  *   the GPU (on different streams, or from different threads) race on the array and
@@ -298,6 +302,39 @@ attn_status attn_get_device_status(void* stream);
  * then reports.  The kernel exits normally; the device stays usable.
  */
 attn_status attn_debug_watchdog(uint64_t timeout_ns, void* stream);
+
+/*
+ * attn_debug_fwd_stall — failure-path check of the prefill kernel (d = 64 or 128).  The
+ * same call as attn_fwd_ex, except that CTA `stall_cta` leaves out its K/V ring fill
+ * number `stall_fill` (0-based, in the order its producer fills the ring) and every
+ * pipeline wait gives up after `timeout_ns` (1 ns .. 10 s) instead of 1 s.  The consumer
+ * of the missing tile waits until its limit runs out, latches ATTN_ERR_DEVICE_TIMEOUT
+ * and raises its CTA's abort flag; every role then winds down (producers wait, bounded,
+ * for their copies in flight, the MMA warp for its MMAs), tensor memory is freed and
+ * the kernel exits.  Other CTAs see the latched status at their next wait and wind down
+ * the same way.  O and lse are then undefined; attn_get_device_status reports the
+ * timeout and the device stays usable.  A stall_fill past the CTA's last fill changes
+ * nothing.  ATTN_ERR_UNSUPPORTED for d = 256.  For testing only.
+ */
+attn_status attn_debug_fwd_stall(const void* q, const void* k, const void* v, void* o,
+                                 int o_dtype, float* lse, int B, int Hq, int Hkv, int Nq,
+                                 int Nk, int d, float scale, int causal, int stall_cta,
+                                 int stall_fill, uint64_t timeout_ns, void* stream);
+
+/*
+ * attn_debug_decode_stall — the same check for the paged decode: attn_decode_paged, with
+ * CTA `stall_cta` of the split kernel leaving out its K/V piece number `stall_piece`
+ * (16 tokens of K and V, in the order its producer gathers them) and pipeline waits
+ * limited to `timeout_ns` (1 ns .. 10 s).  O and lse are then undefined;
+ * attn_get_device_status reports ATTN_ERR_DEVICE_TIMEOUT.  For testing only.
+ */
+attn_status attn_debug_decode_stall(const void* q, const void* k_pool, const void* v_pool,
+                                    const int32_t* block_table, const int32_t* seq_lens,
+                                    int page_size, void* o, float* lse, int num_seqs, int Hq,
+                                    int Hkv, int d, int num_pages, int max_pages_per_seq,
+                                    float scale, void* workspace, size_t workspace_bytes,
+                                    int stall_cta, int stall_piece, uint64_t timeout_ns,
+                                    void* stream);
 
 /*
  * attn_debug_exp2 — evaluates, for i < n, y[i] = 2^x[i] with the polynomial exponential

@@ -193,3 +193,8 @@ def sampled_rows_check(name, n_rows=48, seed_rows=0):
 @pytest.mark.parametrize("name", ["gqa_causal_2k", "gqa_causal_16k", "peaked_mha_d256"])
 def test_full_size_workload_sampled(name, cuda_device):
     sampled_rows_check(name)
+
+
+def test_device_is_sm100(cuda_device):
+    # the library carries sm_100a code only: the device must be compute capability 10.0
+    assert torch.cuda.get_device_capability(cuda_device) == (10, 0)

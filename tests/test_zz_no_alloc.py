@@ -74,3 +74,36 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_device):
     st = lib.attn_decode_paged_noalloc(fake, fake, fake, fake, fake, 16, fake, None, 128, 64, 8, 128, 1000, 2048,
                                        ctypes.c_float(0.1), None)
     assert st == 8 and lib.attn_status_string(st) == b"ATTN_ERR_TOO_LARGE"
+
+
+def _near_limit_pages(lib, S, Hq, Hkv, d, page_size, limit):
+    """Largest max_pages_per_seq, in whole 2048-token work chunks, whose workspace fits."""
+    step = 2048 // page_size
+    pages = step
+    while lib.attn_decode_paged_workspace_size(S, Hq, Hkv, d, pages + step, page_size) <= limit:
+        pages += step
+    return pages
+
+
+def test_noalloc_near_its_limit_matches_workspace_entry(cuda_device):
+    # a call whose scratch layout ends just under the static array's end: the last
+    # sequence uses every page it may, so its partials sit at the far end of the array
+    lib = binding.load_library()
+    limit = lib.attn_decode_paged_noalloc_max_scratch()
+    S, Hq, Hkv, d, ps = 2, 64, 1, 128, 16
+    pages = _near_limit_pages(lib, S, Hq, Hkv, d, ps, limit)
+    need = lib.attn_decode_paged_workspace_size(S, Hq, Hkv, d, pages, ps)
+    assert limit - 2 * (1 << 20) < need <= limit
+    kv = _inputs([1000, pages * ps], Hq=Hq, Hkv=Hkv, d=d, page_size=ps, seed=93, max_pages=pages)
+    _close(*_both(kv, 1.0 / math.sqrt(d)))
+    # one more work chunk per sequence needs more than the array holds: rejected, nothing launched
+    over = pages + 2048 // ps
+    assert lib.attn_decode_paged_workspace_size(S, Hq, Hkv, d, over, ps) > limit
+    dev = torch.device("cuda:0")
+    table = torch.zeros((S, over), dtype=torch.int32, device=dev)
+    o = torch.empty((S, Hq, d), dtype=torch.bfloat16, device=dev)
+    with pytest.raises(ab.AttnError) as e:
+        ab.attn_decode_paged_noalloc(kv.q.to(dev), kv.k_pool.to(dev), kv.v_pool.to(dev), table,
+                                     kv.seq_lens.to(dev), ps, o, None, 0.1)
+    assert e.value.status == 8  # ATTN_ERR_TOO_LARGE
+    assert ab.attn_get_device_status() == 0
