@@ -785,13 +785,14 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
           m = mx;
         }
         const float nmu = (m == -INFINITY) ? 0.0f : -m;
+        // masked blocks take the same path: a hidden key (-inf) comes out of the FMA-pipe
+        // exponential as 2^-125 instead of 0, 2^-100 or less relative to any visible
+        // probability of the row; while the row has seen no visible key (m = -inf) those
+        // values are wiped by the factor 0 at its first visible key, and a row that never
+        // sees one is written as O = 0, LSE = -inf below
         uint32_t P[BN / 2];
         float a0 = 0.f, a1 = 0.f;
-        if (masked) {  // -inf entries: the exp unit returns exact zeros
-          exp_pairs<0u, BN / 2>(s, a.scale_log2, nmu, P, a0, a1);
-        } else {
-          exp_pairs<kEmuMask, BN / 2>(s, a.scale_log2, nmu, P, a0, a1);
-        }
+        exp_pairs<kEmuMask, BN / 2>(s, a.scale_log2, nmu, P, a0, a1);
         l = l * alpha + (a0 + a1);
         // P V of the tile's previous visit (of this unit or the last) must be done: it
         // reads P_t, and O_t may be rescaled.  (Warp-uniform decision: the stores and
@@ -830,6 +831,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_pingpong_kernel(const __grid_
       }
       const bool valid = r < job.rows;
       const size_t row = ((size_t)b * a.Hq + job.hq) * (size_t)a.Nq + (size_t)(valid ? q : 0);
+      if (m == -INFINITY) l = 0.f;  // no visible key: O = 0, LSE = -inf
       if (a.o_f32) {
         store_cols<D>(a, o_addr, have_o, valid, row * D, l);
       } else if (job.rows > quad * 32) {  // the warp has valid rows (warp-uniform)
