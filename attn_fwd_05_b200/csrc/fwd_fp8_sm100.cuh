@@ -464,7 +464,10 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_fp8_kernel(const __grid_const
           float y0, y1, y2, y3, p0, p1, p2, p3;
           fma2(y0, y1, s[4 * i], s[4 * i + 1], c, c, nmu, nmu);
           fma2(y2, y3, s[4 * i + 2], s[4 * i + 3], c, c, nmu, nmu);
-          if (!masked && (i & 3) == 3) {  // a quarter of the pairs on the FMA pipe, as in the bf16 kernel
+          // a quarter of the pairs on the FMA pipe, as in the bf16 kernel; in masked blocks a
+          // hidden key gives 2^-117 (below e4m3's range, so P is 0; a row that never sees a
+          // visible key is written from m = -inf)
+          if ((i & 3) == 3) {
             exp2_fma2(p0, p1, y0, y1);
           } else {
             p0 = ex2(y0);
@@ -524,6 +527,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_fp8_kernel(const __grid_const
       }
       const bool valid = r < job.rows;
       const size_t row = bhq * (size_t)a.Nq + (size_t)(valid ? q : 0);
+      if (m == -INFINITY) l = 0.f;  // no visible key: O = 0, LSE = -inf
       const float sv = __ldg(&a.v_scale[(size_t)b * a.Hkv + kvh]);
       const float inv = l > 0.f ? sv / l : 0.f;  // l already carries the factor 256
       if (!a.o_f32) {
