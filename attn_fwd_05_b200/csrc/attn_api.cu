@@ -16,6 +16,7 @@
 #include "../../include/attn_b200.h"
 #include "backward_sm100.cuh"
 #include "decode_sm100.cuh"
+#include "prefill_d256_sm100.cuh"
 #include "prefill_sm100.cuh"
 #include "fwd_fp8_sm100.cuh"
 

@@ -71,8 +71,8 @@ def parse():
     return p.parse_args()
 
 
-CSRC = ("attn_api.cu", "backward_sm100.cuh", "decode_sm100.cuh", "fwd_fp8_sm100.cuh", "prefill_sm100.cuh",
-        "sm100_common.cuh")
+CSRC = ("attn_api.cu", "backward_sm100.cuh", "decode_sm100.cuh", "fwd_fp8_sm100.cuh", "prefill_d256_sm100.cuh",
+        "prefill_sm100.cuh", "sm100_common.cuh")
 
 
 # the sources each committed ncu summary's kernel is built from (kernel header, shared
@@ -80,7 +80,8 @@ CSRC = ("attn_api.cu", "backward_sm100.cuh", "decode_sm100.cuh", "fwd_fp8_sm100.
 PROFILE_SOURCES = {
     "attn_fwd_pingpong_gqa_causal_2k.md": ("attn_api.cu", "prefill_sm100.cuh", "sm100_common.cuh"),
     "attn_fwd_pingpong_gqa_causal_16k.md": ("attn_api.cu", "prefill_sm100.cuh", "sm100_common.cuh"),
-    "attn_fwd_single_peaked_mha_d256.md": ("attn_api.cu", "prefill_sm100.cuh", "sm100_common.cuh"),
+    "attn_fwd_single_peaked_mha_d256.md": ("attn_api.cu", "prefill_d256_sm100.cuh", "prefill_sm100.cuh",
+                                           "sm100_common.cuh"),
     "attn_decode_split_paged_decode.md": ("attn_api.cu", "decode_sm100.cuh", "sm100_common.cuh"),
     "attn_bwd_gqa_causal_2k.md": ("attn_api.cu", "backward_sm100.cuh", "sm100_common.cuh"),
     "attn_fwd_fp8_gqa_causal_2k.md": ("attn_api.cu", "fwd_fp8_sm100.cuh", "sm100_common.cuh"),
@@ -429,41 +430,16 @@ def config_block(args, shape):
     return cfg
 
 
-def run_backward(args, dist):
-    """Backward pass (attn_bwd: delta, dK/dV and dQ kernels) on a prefill workload.  FLOPs are
-    the method's five products, 2.5x the forward's (causal halved), as the pages' FA figures
-    count them; the dQ kernel's recomputation of S and dP is not counted."""
-    import attn_fwd_05_b200 as ab
-    ab.load_library()
-    dev = torch.device("cuda", dist.local)
-    torch.cuda.set_device(dev)
-    peaks, peak_src = load_peaks()
-    name = args.workload[: -len("_bwd")]
-    shape = synth.WORKLOADS[name]
-    seed = rank_seed(synth.workload_seed(name), dist.rank)
-    pre = make_prefill(shape, seed, dev)
-    qd, kd, vd = pre["dev"]
-    do = synth.upstream_grad(shape, seed).to(dev)
-    scale = synth.default_scale(shape.d)
-    stream = torch.cuda.current_stream(dev)
-    ab.attn_fwd(qd, kd, vd, pre["o"], pre["lse"], shape.causal, scale, stream)
-    dq = torch.empty((shape.B, shape.Hq, shape.Nq, shape.d), dtype=torch.float32, device=dev)
-    dk = torch.empty((shape.B, shape.Hkv, shape.Nk, shape.d), dtype=torch.float32, device=dev)
-    dv = torch.empty_like(dk)
-    ws = torch.empty(ab.attn_bwd_workspace_size(shape.B, shape.Hq, shape.Nq), dtype=torch.uint8, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    flops = 2.5 * counts.prefill_flops(shape.B, shape.Hq, shape.Nq, shape.Nk, shape.d, shape.causal)
-
-    def step():
-        ab.attn_bwd(qd, kd, vd, pre["o"], do, pre["lse"], dq, dk, dv, shape.causal, scale, ws, stream)
-
+def timed_launches(step, K, W, flush, stream, dist, dev):
+    """W untimed calls, then K calls each after an L2 flush, each bracketed by CUDA events on
+    the launching stream (barrier and synchronize on both sides); the clocks are sampled
+    throughout.  Returns the per-call milliseconds and the clock record."""
     clocks = ClockSampler(dist.local)
     clocks.start()
-    for _ in range(args.warmup):
+    for _ in range(W):
         step()
         flush.zero_()
     torch.cuda.synchronize(dev)
-    K = args.steps
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K)]
     dist.barrier()
     torch.cuda.synchronize(dev)
@@ -475,34 +451,141 @@ def run_backward(args, dist):
     torch.cuda.synchronize(dev)
     dist.barrier()
     clk = clocks.stop()
+    return [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K)], clk
+
+
+def bwd_record(args, ab, name, dev, stream, dist, peaks, peak_src, K, W, cpu=True):
+    """Backward pass (attn_bwd: delta, dK/dV and dQ kernels) of a prefill workload.  FLOPs are
+    the method's five products, 2.5x the forward's (causal halved), as the pages' FA figures
+    count them; the dQ kernel's recomputation of S and dP is not counted."""
+    shape = synth.WORKLOADS[name]
+    seed = rank_seed(synth.workload_seed(name), dist.rank)
+    pre = make_prefill(shape, seed, dev)
+    qd, kd, vd = pre["dev"]
+    do = synth.upstream_grad(shape, seed).to(dev)
+    scale = synth.default_scale(shape.d)
+    ab.attn_fwd(qd, kd, vd, pre["o"], pre["lse"], shape.causal, scale, stream)
+    dq = torch.empty((shape.B, shape.Hq, shape.Nq, shape.d), dtype=torch.float32, device=dev)
+    dk = torch.empty((shape.B, shape.Hkv, shape.Nk, shape.d), dtype=torch.float32, device=dev)
+    dv = torch.empty_like(dk)
+    ws = torch.empty(ab.attn_bwd_workspace_size(shape.B, shape.Hq, shape.Nq), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flops = 2.5 * counts.prefill_flops(shape.B, shape.Hq, shape.Nq, shape.Nk, shape.d, shape.causal)
+
+    def step():
+        ab.attn_bwd(qd, kd, vd, pre["o"], do, pre["lse"], dq, dk, dv, shape.causal, scale, ws, stream)
+
+    ms, clk = timed_launches(step, K, W, flush, stream, dist, dev)
     st = ab.attn_get_device_status(stream)
     if st != 0:
         raise RuntimeError(f"kernel fault in the timed region: {ab.attn_status_string(st)}")
-    ms = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K)]
     tot = dist.max(sum(ms))
     achieved = flops / (sum(ms) / K * 1e-3) / 1e12
-    line = {
-        "metric": "attn bwd TFLOPS & % of BF16 tensor peak", "value": dist.world * flops * K / (tot * 1e-3) / 1e12,
-        "unit": "TFLOP/s", "n_gpus": dist.world, "steps": K, "warmup": args.warmup, "ms_per_step": tot / K,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload,
-                   "prefill": {"B": shape.B, "Hq": shape.Hq, "Hkv": shape.Hkv, "Nq": shape.Nq, "Nk": shape.Nk,
-                               "d": shape.d, "causal": shape.causal},
-                   "l2": "L2 flushed between steps by writing a 256 MB buffer",
-                   "parallelism": f"independent replicas x{dist.world} (no data-path collective)"},
+    rec = {
+        "metric": "attn bwd TFLOPS & % of BF16 tensor peak", "unit": "TFLOP/s",
+        "value": dist.world * flops * K / (tot * 1e-3) / 1e12, "steps": K, "ms_per_launch": tot / K,
+        "median_ms": statistics.median(ms),
+        "shape": {"B": shape.B, "Hq": shape.Hq, "Hkv": shape.Hkv, "Nq": shape.Nq, "Nk": shape.Nk, "d": shape.d,
+                  "causal": shape.causal},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_tflops"],
                      "traffic": profiled_traffic(f"attn_bwd_{name}.md") if name in ("gqa_causal_2k", "gqa_causal_16k")
                      else None,
                      "peak_source": f"{peak_src} bf16_tflops (burst cuBLAS)",
                      "kernel": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel + attn_bwd_delta_kernel (one call)",
-                     "flops_per_launch": flops, "median_ms": statistics.median(ms)},
-        "gpu_launches": 3 * K, "clocks": clk,
+                     "flops_per_launch": flops},
+        "l2": "L2 flushed before every call by writing a 256 MB buffer",
+        "clocks": clk, "gpu_launches": 3 * K,
     }
-    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_backward_sample(shape, pre["host"], do.cpu(), scale, flops, args.cpu_seconds)
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline and cpu:
+        rec["cpu_baseline"] = oracle_backward_sample(shape, pre["host"], do.cpu(), scale, flops, args.cpu_seconds / 2)
+    return rec
+
+
+def fp8_record(args, ab, name, dev, stream, dist, peaks, peak_src, K, W, cpu=True):
+    """FP8 forward (attn_fwd_fp8) of a d = 128 prefill workload: inputs quantized on the GPU
+    once (Q, K per 128 rows, V per head), outside the timed region.  The tensor peak for
+    e4m3 is the measured bf16 figure times the nominal dense ratio 4.5 / 2.25 = 2."""
+    shape = synth.WORKLOADS[name]
+    seed = rank_seed(synth.workload_seed(name), dist.rank)
+    pre = make_prefill(shape, seed, dev)
+    qd, kd, vd = pre["dev"]
+    q8, qs = ab.attn_quantize_fp8(qd, 128)
+    k8, ks = ab.attn_quantize_fp8(kd, 128)
+    v8, vs = ab.attn_quantize_fp8(vd, shape.Nk)
+    vs = vs[..., 0].contiguous()
+    scale = synth.default_scale(shape.d)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flops = counts.prefill_flops(shape.B, shape.Hq, shape.Nq, shape.Nk, shape.d, shape.causal)
+
+    def step():
+        ab.attn_fwd_fp8(q8, qs, k8, ks, v8, vs, pre["o"], pre["lse"], shape.causal, scale, stream)
+
+    ms, clk = timed_launches(step, K, W, flush, stream, dist, dev)
+    st = ab.attn_get_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"kernel fault in the timed region: {ab.attn_status_string(st)}")
+    tot = dist.max(sum(ms))
+    achieved = flops / (sum(ms) / K * 1e-3) / 1e12
+    peak = 2.0 * peaks["bf16_tflops"]
+    rec = {
+        "metric": "attn fwd TFLOPS (e4m3 inputs) & % of FP8 tensor peak", "unit": "TFLOP/s",
+        "value": dist.world * flops * K / (tot * 1e-3) / 1e12, "steps": K, "ms_per_launch": tot / K,
+        "median_ms": statistics.median(ms), "dtype": "e4m3 (fp32 accumulate)",
+        "shape": {"B": shape.B, "Hq": shape.Hq, "Hkv": shape.Hkv, "Nq": shape.Nq, "Nk": shape.Nk, "d": shape.d,
+                  "causal": shape.causal},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak,
+                     "traffic": profiled_traffic(f"attn_fwd_fp8_{name}.md")
+                     if name in ("gqa_causal_2k", "gqa_causal_16k") else None,
+                     "peak_source": f"2 x {peak_src} bf16_tflops (nominal e4m3 : bf16 dense ratio)",
+                     "kernel": "attn_fwd_fp8_kernel", "flops_per_launch": flops},
+        "l2": "L2 flushed before every launch by writing a 256 MB buffer",
+        "clocks": clk, "gpu_launches": K,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline and cpu:
+        import oracle
+        q, k, v = pre["host"]
+        q8h, qsh = oracle.block_quantize(q, 128)
+        k8h, ksh = oracle.block_quantize(k, 128)
+        v8h, vsh = oracle.block_quantize(v, shape.Nk)
+        qdq = torch.from_numpy(oracle.dequantize(q8h, qsh))
+        kdq = torch.from_numpy(oracle.dequantize(k8h, ksh))
+        vdq = torch.from_numpy(oracle.dequantize(v8h, vsh, block=shape.Nk))
+        rec["cpu_baseline"] = oracle_prefill_sample(shape, qdq, kdq, vdq, args.cpu_seconds / 2)
+        rec["cpu_baseline"]["sample"] += " (exact attention of the dequantized e4m3 inputs)"
+    return rec
+
+
+def variant_line(args, dist, rec, workload):
+    """The JSON line of a --workload *_bwd / *_fp8 run, built from its record."""
+    shape = rec["shape"]
+    line = {
+        "metric": rec["metric"], "value": rec["value"], "unit": rec["unit"], "n_gpus": dist.world,
+        "steps": rec["steps"], "warmup": args.warmup, "ms_per_step": rec["ms_per_launch"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": rec.get("dtype", "bf16"),
+        "data": "synthetic",
+        "config": {"workload": workload, "prefill": shape, "l2": rec["l2"],
+                   "parallelism": f"independent replicas x{dist.world} (no data-path collective)"},
+        "roofline": dict(rec["roofline"], median_ms=rec["median_ms"]),
+        "gpu_launches": rec["gpu_launches"], "clocks": rec["clocks"],
+    }
+    if "cpu_baseline" in rec:
+        line["cpu_baseline"] = rec["cpu_baseline"]
+    return line
+
+
+def run_backward(args, dist):
+    import attn_fwd_05_b200 as ab
+    ab.load_library()
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    rec = bwd_record(args, ab, args.workload[: -len("_bwd")], dev, stream, dist, peaks, peak_src, args.steps,
+                     args.warmup)
     if dist.rank == 0:
-        print(json.dumps(line), flush=True)
+        print(json.dumps(variant_line(args, dist, rec, args.workload)), flush=True)
     return 0
 
 
@@ -541,76 +624,16 @@ def oracle_backward_sample(shape, host, do, scale, flops, seconds):
 
 
 def run_fp8(args, dist):
-    """FP8 forward (attn_fwd_fp8) on a d = 128 prefill workload: inputs quantized on the GPU
-    once (Q, K per 128 rows, V per head), outside the timed region.  The tensor peak for
-    e4m3 is the measured bf16 figure times the nominal dense ratio 4.5 / 2.25 = 2."""
     import attn_fwd_05_b200 as ab
     ab.load_library()
     dev = torch.device("cuda", dist.local)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
-    name = args.workload[: -len("_fp8")]
-    shape = synth.WORKLOADS[name]
-    seed = rank_seed(synth.workload_seed(name), dist.rank)
-    pre = make_prefill(shape, seed, dev)
-    qd, kd, vd = pre["dev"]
-    q8, qs = ab.attn_quantize_fp8(qd, 128)
-    k8, ks = ab.attn_quantize_fp8(kd, 128)
-    v8, vs = ab.attn_quantize_fp8(vd, shape.Nk)
-    vs = vs[..., 0].contiguous()
-    scale = synth.default_scale(shape.d)
     stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    flops = counts.prefill_flops(shape.B, shape.Hq, shape.Nq, shape.Nk, shape.d, shape.causal)
-
-    def step():
-        ab.attn_fwd_fp8(q8, qs, k8, ks, v8, vs, pre["o"], pre["lse"], shape.causal, scale, stream)
-
-    clocks = ClockSampler(dist.local)
-    clocks.start()
-    for _ in range(args.warmup):
-        step()
-        flush.zero_()
-    torch.cuda.synchronize(dev)
-    K = args.steps
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K)]
-    dist.barrier()
-    torch.cuda.synchronize(dev)
-    for i in range(K):
-        flush.zero_()
-        ev[2 * i].record(stream)
-        step()
-        ev[2 * i + 1].record(stream)
-    torch.cuda.synchronize(dev)
-    dist.barrier()
-    clk = clocks.stop()
-    st = ab.attn_get_device_status(stream)
-    if st != 0:
-        raise RuntimeError(f"kernel fault in the timed region: {ab.attn_status_string(st)}")
-    ms = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K)]
-    tot = dist.max(sum(ms))
-    achieved = flops / (sum(ms) / K * 1e-3) / 1e12
-    peak = 2.0 * peaks["bf16_tflops"]
-    line = {
-        "metric": "attn fwd TFLOPS (e4m3 inputs) & % of FP8 tensor peak",
-        "value": dist.world * flops * K / (tot * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": dist.world,
-        "steps": K, "warmup": args.warmup, "ms_per_step": tot / K, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)", "data": "synthetic",
-        "config": {"workload": args.workload,
-                   "prefill": {"B": shape.B, "Hq": shape.Hq, "Hkv": shape.Hkv, "Nq": shape.Nq, "Nk": shape.Nk,
-                               "d": shape.d, "causal": shape.causal},
-                   "l2": "L2 flushed between steps by writing a 256 MB buffer",
-                   "parallelism": f"independent replicas x{dist.world} (no data-path collective)"},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak,
-                     "traffic": profiled_traffic(f"attn_fwd_fp8_{args.workload[:-len('_fp8')]}.md")
-                     if args.workload in ("gqa_causal_2k_fp8", "gqa_causal_16k_fp8") else None,
-                     "peak_source": f"2 x {peak_src} bf16_tflops (nominal e4m3 : bf16 dense ratio)",
-                     "kernel": "attn_fwd_fp8_kernel", "flops_per_launch": flops, "median_ms": statistics.median(ms)},
-        "gpu_launches": K, "clocks": clk,
-    }
+    rec = fp8_record(args, ab, args.workload[: -len("_fp8")], dev, stream, dist, peaks, peak_src, args.steps,
+                     args.warmup)
     if dist.rank == 0:
-        print(json.dumps(line), flush=True)
+        print(json.dumps(variant_line(args, dist, rec, args.workload)), flush=True)
     return 0
 
 
@@ -749,6 +772,16 @@ def run_ours(args, dist):
         torch.cuda.empty_cache()
         line["workloads"] = {name: prefill_record(args, ab, name, dev, stream, dist, peaks, peak_src)
                              for name in OTHER_PREFILL}
+        # the backward pass and the FP8 forward of the two GQA causal workloads
+        # (CPU baselines for the 2K variants only: one 16K head of the fp64 backward oracle
+        # takes minutes on one thread, and the 16K forward's oracle rate is in its own record)
+        for name in ("gqa_causal_2k", "gqa_causal_16k"):
+            small = name == "gqa_causal_2k"
+            K = max(3, min(args.steps, 20 if small else 8))
+            line["workloads"][name + "_fp8"] = fp8_record(args, ab, name, dev, stream, dist, peaks, peak_src, K,
+                                                          max(3, args.warmup), cpu=small)
+            line["workloads"][name + "_bwd"] = bwd_record(args, ab, name, dev, stream, dist, peaks, peak_src, K,
+                                                          max(3, args.warmup), cpu=small)
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     return 0
