@@ -12,7 +12,9 @@ prefill launch starts with a cold L2 for its own inputs.
 Printed (rank 0, one JSON line): prefill TFLOP/s as `value` (causal FLOPs counted as
 half of 4*B*Hq*Nq*Nk*d), the decode KV-read GB/s in `decode`, roofline fractions
 against MEASURED_PEAKS.json, the end-to-end figures through the public API with host
-buffers (`e2e` for the prefill, `decode.e2e` for the decode), the fp64 CPU oracle timed
+buffers (`e2e` for the prefill, `decode.e2e` for the decode; two buffer slots overlap
+the copies of neighbouring steps with the kernel, and the back-to-back figure is kept
+beside it as `sequential`), the fp64 CPU oracle timed
 on a bounded sample (`cpu_baseline`), and the SM clocks sampled during the run.  After
 the timed step, the other prefill configurations (the tiny d=64 case, the 16K
 long-context case and the peaked d=256 case) are each timed on their own, L2 flushed
@@ -853,86 +855,150 @@ def prefill_record(args, ab, name, dev, stream, dist, peaks, peak_src):
     return rec
 
 
+def _pipelined_e2e(K, h2d, launch, d2h, stream, dev, dist, slots=2):
+    """Time K steps of (copy in, launch, copy out) as a serving loop runs them: two slots of
+    device buffers, the host-to-device copies on one stream, the kernels on the caller's
+    stream and the device-to-host copies on a third, so step i+1's inputs go up and step
+    i-1's outputs come down while step i computes (PCIe is full duplex).  Events order each
+    slot's reuse: a copy into slot j waits for the kernel that last read it, a kernel
+    writing slot j waits for the copy that last read its outputs.  The timed region starts
+    before the first copy in and ends after the last copy out.  Returns the max over ranks
+    of the region's milliseconds."""
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    in_done = [torch.cuda.Event() for _ in range(slots)]
+    comp_done = [torch.cuda.Event() for _ in range(slots)]
+    out_done = [torch.cuda.Event() for _ in range(slots)]
+
+    def step(i):
+        j = i % slots
+        s_in.wait_event(comp_done[j])  # no-op until the event is first recorded
+        with torch.cuda.stream(s_in):
+            h2d(j)
+        in_done[j].record(s_in)
+        stream.wait_event(in_done[j])
+        stream.wait_event(out_done[j])
+        launch(j)
+        comp_done[j].record(stream)
+        s_out.wait_event(comp_done[j])
+        with torch.cuda.stream(s_out):
+            d2h(j)
+        out_done[j].record(s_out)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    a.record(stream)
+    s_in.wait_event(a)
+    for i in range(K):
+        step(i)
+    for e in out_done:
+        stream.wait_event(e)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    return dist.max(a.elapsed_time(b))
+
+
+def _sequential_e2e(K, h2d, launch, d2h, stream, dev, dist):
+    """K steps of (copy in, launch, copy out), all on the caller's stream, one after the
+    other.  Returns the max over ranks of the timed region's milliseconds."""
+    def step():
+        with torch.cuda.stream(stream):
+            h2d(0)
+            launch(0)
+            d2h(0)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    a.record(stream)
+    for _ in range(K):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    return dist.max(a.elapsed_time(b))
+
+
 def e2e_decode(args, ab, dec, scale, dev, stream, dist):
     """The decode metric through the public API with host buffers: every step copies the
     step's inputs (the query tokens, the block table and the sequence lengths) from
     pinned host memory, runs attn_decode_paged, and copies O and LSE back, all inside the
     timed region.  The paged K/V pools are the cache: they stay resident in HBM across
-    steps, as a serving engine keeps them."""
-    qh = dec["kv"].q.pin_memory()
-    th = dec["kv"].block_table.pin_memory()
-    lh = dec["kv"].seq_lens.pin_memory()
-    oh = torch.empty(dec["o"].shape, dtype=torch.bfloat16).pin_memory()
-    lseh = torch.empty(dec["lse"].shape, dtype=torch.float32).pin_memory()
-    qd = torch.empty_like(qh, device=dev)
-    td = torch.empty_like(th, device=dev)
-    ld = torch.empty_like(lh, device=dev)
+    steps, as a serving engine keeps them.  The headline value overlaps the copies of
+    neighbouring steps with the kernel (two buffer slots); the sequential figure runs
+    copy, kernel and copy back to back."""
+    hin = [t.pin_memory() for t in (dec["kv"].q, dec["kv"].block_table, dec["kv"].seq_lens)]
+    din = [[torch.empty_like(t, device=dev) for t in hin] for _ in range(2)]
+    dout = [(torch.empty_like(dec["o"]), torch.empty_like(dec["lse"])) for _ in range(2)]
+    hout = [(torch.empty(dec["o"].shape, dtype=torch.bfloat16).pin_memory(),
+             torch.empty(dec["lse"].shape, dtype=torch.float32).pin_memory()) for _ in range(2)]
 
-    def step():
-        qd.copy_(qh, non_blocking=True)
-        td.copy_(th, non_blocking=True)
-        ld.copy_(lh, non_blocking=True)
-        ab.attn_decode_paged(qd, dec["k_pool"], dec["v_pool"], td, ld, dec["shape"].page_size, dec["o"], dec["lse"],
-                             scale, dec["ws"], stream)
-        oh.copy_(dec["o"], non_blocking=True)
-        lseh.copy_(dec["lse"], non_blocking=True)
+    def h2d(j):
+        for d, h in zip(din[j], hin):
+            d.copy_(h, non_blocking=True)
+
+    def launch(j):
+        qd, td, ld = din[j]
+        ab.attn_decode_paged(qd, dec["k_pool"], dec["v_pool"], td, ld, dec["shape"].page_size, dout[j][0],
+                             dout[j][1], scale, dec["ws"], stream)
+
+    def d2h(j):
+        for h, d in zip(hout[j], dout[j]):
+            h.copy_(d, non_blocking=True)
 
     K = max(3, min(args.steps, 20))
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize(dev)
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    dist.barrier()
-    a.record(stream)
-    for _ in range(K):
-        step()
-    b.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = dist.max(a.elapsed_time(b))
-    h2d = sum(t.numel() * t.element_size() for t in (qh, th, lh))
-    d2h = oh.numel() * 2 + lseh.numel() * 4
-    return {"value": dist.world * dec["kv_bytes"] * K / (ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": K,
+    ms = _pipelined_e2e(K, h2d, launch, d2h, stream, dev, dist)
+    seq_ms = _sequential_e2e(K, h2d, launch, d2h, stream, dev, dist)
+    h2d_b = sum(t.numel() * t.element_size() for t in hin)
+    d2h_b = sum(t.numel() * t.element_size() for t in hout[0])
+    rate = dist.world * dec["kv_bytes"] * K / 1e9
+    return {"value": rate / (ms * 1e-3), "unit": "GB/s", "h2d_bytes_per_step": h2d_b,
+            "d2h_bytes_per_step": d2h_b, "steps": K, "ms_per_step": ms / K,
+            "sequential": {"value": rate / (seq_ms * 1e-3), "ms_per_step": seq_ms / K},
             "note": "paged K/V pools resident in HBM (the cache); query, block table and lengths copied in, "
-                    "O and LSE copied out every step"}
+                    "O and LSE copied out every step; two buffer slots, copies of neighbouring steps "
+                    "overlap the kernel (sequential: copy, kernel, copy back to back)"}
 
 
 def e2e_prefill(args, ab, pre, shape, scale, flops, dev, stream, dist):
-    """Same metric through the public API with host buffers: H2D of q, k, v from pinned
-    memory, attn_fwd, D2H of o and lse, all inside the timed region."""
-    qh, kh, vh = (t.pin_memory() for t in pre["host"])
-    oh = torch.empty(pre["o"].shape, dtype=torch.bfloat16).pin_memory()
-    lh = torch.empty(pre["lse"].shape, dtype=torch.float32).pin_memory()
-    qd = torch.empty_like(qh, device=dev)
-    kd = torch.empty_like(kh, device=dev)
-    vd = torch.empty_like(vh, device=dev)
+    """Same metric through the public API with host buffers: every step copies q, k, v in
+    from pinned memory, runs attn_fwd and copies o and lse out, all inside the timed
+    region.  The headline value overlaps the copies of neighbouring steps with the kernel
+    (two buffer slots); the sequential figure runs copy, kernel and copy back to back."""
+    hin = [t.pin_memory() for t in pre["host"]]
+    din = [[torch.empty_like(t, device=dev) for t in hin] for _ in range(2)]
+    dout = [(torch.empty_like(pre["o"]), torch.empty_like(pre["lse"])) for _ in range(2)]
+    hout = [(torch.empty(pre["o"].shape, dtype=torch.bfloat16).pin_memory(),
+             torch.empty(pre["lse"].shape, dtype=torch.float32).pin_memory()) for _ in range(2)]
 
-    def step():
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        ab.attn_fwd(qd, kd, vd, pre["o"], pre["lse"], shape.causal, scale, stream)
-        oh.copy_(pre["o"], non_blocking=True)
-        lh.copy_(pre["lse"], non_blocking=True)
+    def h2d(j):
+        for d, h in zip(din[j], hin):
+            d.copy_(h, non_blocking=True)
+
+    def launch(j):
+        ab.attn_fwd(*din[j], dout[j][0], dout[j][1], shape.causal, scale, stream)
+
+    def d2h(j):
+        for h, d in zip(hout[j], dout[j]):
+            h.copy_(d, non_blocking=True)
 
     K = max(3, min(args.steps, 20))
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize(dev)
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    dist.barrier()
-    a.record(stream)
-    for _ in range(K):
-        step()
-    b.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = dist.max(a.elapsed_time(b))
-    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
-    d2h = oh.numel() * 2 + lh.numel() * 4
-    return {"value": dist.world * flops * K / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K}
+    ms = _pipelined_e2e(K, h2d, launch, d2h, stream, dev, dist)
+    seq_ms = _sequential_e2e(K, h2d, launch, d2h, stream, dev, dist)
+    h2d_b = sum(t.numel() * t.element_size() for t in hin)
+    d2h_b = sum(t.numel() * t.element_size() for t in hout[0])
+    rate = dist.world * flops * K / 1e12
+    return {"value": rate / (ms * 1e-3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d_b,
+            "d2h_bytes_per_step": d2h_b, "steps": K, "ms_per_step": ms / K,
+            "sequential": {"value": rate / (seq_ms * 1e-3), "ms_per_step": seq_ms / K},
+            "note": "two buffer slots: step i+1's copy in and step i-1's copy out overlap step i's kernel "
+                    "(sequential: copy, kernel, copy back to back)"}
 
 
 def main():
