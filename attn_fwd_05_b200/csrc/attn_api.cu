@@ -112,41 +112,6 @@ bool ensure_smem(K kernel, int bytes, int slot) {
   return true;
 }
 
-// A second stream per device for the dQ kernel of attn_bwd, and the events that fork it
-// from the caller's stream and join it back (created on first use).  Callers hold
-// side_mutex() from the fork to the join, so concurrent calls do not interleave their
-// records and waits.
-struct SideStream {
-  cudaStream_t stream = nullptr;
-  cudaEvent_t fork = nullptr;
-  cudaEvent_t join = nullptr;
-};
-
-std::mutex& side_mutex() {
-  static std::mutex mu;
-  return mu;
-}
-
-// The current device's side stream, or nullptr if it could not be created (the caller
-// then stays on its own stream).  Call with side_mutex() held.
-SideStream* side_stream() {
-  static SideStream ss[kMaxDevices];
-  static bool failed[kMaxDevices] = {};
-  const int dev = current_device();
-  if (dev < 0 || dev >= kMaxDevices || failed[dev]) return nullptr;
-  SideStream& s = ss[dev];
-  if (s.stream == nullptr) {
-    if (cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess) {
-      cudaGetLastError();
-      failed[dev] = true;
-      return nullptr;
-    }
-  }
-  return &s;
-}
-
 int sm_count() {
   static std::atomic<int> cache[kMaxDevices];
   const int dev = current_device();
@@ -195,33 +160,16 @@ attn_status launch_bwd(attn::BwdArgs& a, const void* o, const void* dout, float*
   using C = attn::BwdCfg<D>;
   const long long rows = (long long)a.B * a.Hq * a.Nq;
   const long long dblocks = std::min<long long>((rows + 7) / 8, (long long)sm_count() * 16);
-  auto kkv = attn::attn_bwd_dkdv_kernel<D>;
-  auto kq = attn::attn_bwd_dq_kernel<D>;
-  const int slot = D == 64 ? 9 : 10;  // shared-memory slots 9-12: backward kernels
-  if (!ensure_smem(kkv, C::SMEM, slot) || !ensure_smem(kq, C::SMEM, slot + 2)) return ATTN_ERR_CUDA;
-  const long long gkv = (long long)a.B * a.Hkv * a.n_ktiles;
-  const long long gq = (long long)a.B * a.Hq * a.n_qtiles;
-  if (gkv > 0x7fffffffLL || gq > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  auto k = attn::attn_bwd_kernel<D>;
+  const int slot = D == 64 ? 9 : 10;  // shared-memory slots 9-10: backward kernels
+  if (!ensure_smem(k, C::SMEM, slot)) return ATTN_ERR_CUDA;
+  const long long grid = (long long)a.B * a.Hkv * a.n_ktiles;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  // Delta, and dQ cleared for the main kernel's reduce-adds
   attn::attn_bwd_delta_kernel<D><<<(unsigned)dblocks, 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), delta, rows);
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), delta, a.dq, rows);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  // dK/dV and dQ need only Delta and the inputs: the dQ kernel runs on a side stream
-  // forked after Delta and joined before the call returns, so its CTAs fill the SMs the
-  // dK/dV kernel's last wave leaves free
-  std::lock_guard<std::mutex> g(side_mutex());
-  SideStream* side = side_stream();
-  if (side != nullptr && cudaEventRecord(side->fork, st) != cudaSuccess) return ATTN_ERR_CUDA;
-  kkv<<<(unsigned)gkv, C::THREADS, C::SMEM, st>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  if (side == nullptr) {
-    kq<<<(unsigned)gq, C::THREADS, C::SMEM, st>>>(a);
-    return launch_status();
-  }
-  if (cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess) return ATTN_ERR_CUDA;
-  kq<<<(unsigned)gq, C::THREADS, C::SMEM, side->stream>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  if (cudaEventRecord(side->join, side->stream) != cudaSuccess || cudaStreamWaitEvent(st, side->join, 0) != cudaSuccess)
-    return ATTN_ERR_CUDA;
+  k<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(a);
   return launch_status();
 }
 

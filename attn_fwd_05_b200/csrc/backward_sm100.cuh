@@ -7,20 +7,23 @@
 // Delta = rowsum(dO o O):
 //     dV = P^T dO,  dP = dO V^T,  dS = P o (dP - Delta),  dQ = scale dS K,  dK = scale dS^T Q.
 //
-// B200 design: three kernels, no atomics.
-//   * delta kernel: one warp per query row, Delta in fp32.
-//   * dK/dV kernel: one CTA per (batch, KV head, 128-key tile).  It walks the query
-//     heads of the KV head's group and the q-tiles that see its keys, and keeps dK and
-//     dV for its keys in TMEM for the whole walk (the group's sum comes for free):
-//     S^T = K Q^T and dP^T = V dO^T land in TMEM (one thread per key row), the thread
-//     writes P^T and dS^T back over them as bf16, and dV += P^T dO, dK += dS^T Q run
-//     with A from TMEM.  Q and dO tiles stream through a two-stage TMA ring.
-//   * dQ kernel: one CTA per (batch, query head, 128-row q-tile).  It walks the K/V
-//     tiles its rows see: S = Q K^T and dP = dO V^T in TMEM (one thread per query row),
-//     dS written back over S, dQ += dS K with A from TMEM.
-//   S and dP are computed by both kernels (the dQ pass repeats two of the five
-//   products) in exchange for no atomic accumulation.
-//   TMEM per CTA: S, dP (128 columns each) and the accumulators (d columns each).
+// B200 design: one pass over the score matrix, five products per block.
+//   * delta kernel: one warp per query row, Delta in fp32; it also clears the row of dQ
+//     that the main kernel accumulates into.
+//   * main kernel: one CTA per (batch, KV head, 128-key tile), longest first under the
+//     causal mask.  It walks the query heads of the KV head's group and the q-tiles that
+//     see its keys (a step = one 128-query tile of one head) and keeps dK and dV for its
+//     keys in TMEM for the whole walk, so the group's sum needs no atomics.  Per step:
+//       S^T = K Q^T and dP^T = V dO^T land in TMEM (128 x 128 each, one key row per TMEM
+//       lane); the elementwise warps turn S^T into P^T (bf16, written back over S^T) and
+//       dP^T into dS^T (bf16, to shared memory in the 128-byte swizzled layout);
+//       dV += P^T dO takes A from TMEM; dK += dS^T Q reads dS^T K-major; dQ_step = dS K
+//       reads the same shared dS^T MN-major, into TMEM.  A drain warpgroup moves dQ_step
+//       out of TMEM, scales it and adds it to the global dQ with TMA reduce-adds (fp32,
+//       performed in L2), staged in the ring stage the step has finished with.
+//   TMEM (512 columns): S^T, dP^T (128 each), dV and dK (d each).  At d = 128 dQ_step
+//   takes the dP^T columns once the elementwise pass has read them; at d = 64 it has
+//   columns of its own.
 // Causal masking uses the forward's bottom-right alignment: key j is visible to query i
 // iff j <= i + (Nk - Nq).  d = 64 or 128.
 #pragma once
@@ -34,12 +37,12 @@ struct BwdArgs {
   CUtensorMap tm_do;  // same layout as Q
   CUtensorMap tm_k;   // [B*Hkv, Nk, d] bf16, box {64, 128, 1}
   CUtensorMap tm_v;
-  CUtensorMap tm_dq;   // fp32 [B*Hq, Nq, d], box {32, 32, 1}: the gradients leave through TMA stores
-  CUtensorMap tm_dk;   // fp32 [B*Hkv, Nk, d], same boxes
+  CUtensorMap tm_dq;   // fp32 [B*Hq, Nq, d], box {32, 32, 1}: dQ is accumulated by TMA reduce-adds
+  CUtensorMap tm_dk;   // fp32 [B*Hkv, Nk, d], same boxes, written by TMA stores
   CUtensorMap tm_dv;
   const float* lse;    // [B*Hq, Nq] natural log-sum-exp of the forward pass
   const float* delta;  // [B*Hq, Nq] rowsum(dO o O)
-  float* dq;           // [B*Hq, Nq, d]
+  float* dq;           // [B*Hq, Nq, d], cleared by the delta kernel
   float* dk;           // [B*Hkv, Nk, d]
   float* dv;           // [B*Hkv, Nk, d]
   int B, Hq, Hkv, Nq, Nk, group, causal, n_qtiles, n_ktiles;
@@ -60,7 +63,8 @@ __device__ __forceinline__ float lse2_of(const BwdArgs& a, size_t bh, int q) {
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const __nv_bfloat16* __restrict__ o,
                                                              const __nv_bfloat16* __restrict__ dout,
-                                                             float* __restrict__ delta, long long rows) {
+                                                             float* __restrict__ delta, float* __restrict__ dq,
+                                                             long long rows) {
   const int lane = threadIdx.x & 31;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
   for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows; r += nwarps) {
@@ -73,6 +77,9 @@ __global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const __nv_bfloat16
       const float2 y = __bfloat1622float2(pd[c]);
       acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
     }
+    float4* z = reinterpret_cast<float4*>(dq + r * D);
+#pragma unroll
+    for (int c = lane; c < D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
     if (lane == 0) delta[r] = acc;
@@ -80,51 +87,6 @@ __global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const __nv_bfloat16
 }
 
 // ------------------------------------------------------------------- shared pieces
-
-// One 32-column chunk of a probability / gradient row: p = 2^(s sl2 - L2) where the
-// column is visible, ds = p (dp - dl); both packed to bf16 pairs.
-__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], float sl2,
-                                          const float* L2, const float* dl, int vis_lo, int vis_hi, uint32_t (&P)[16],
-                                          uint32_t (&dS)[16]) {
-#pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    float p[2], g[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int c = i + e;
-      const bool vis = c >= vis_lo && c <= vis_hi;
-      const float y = fmaf(__uint_as_float(s[c]), sl2, -L2[c]);
-      p[e] = vis ? ex2(y) : 0.f;
-      g[e] = p[e] * (__uint_as_float(dp[c]) - dl[c]);
-    }
-    P[i / 2] = pack_bf16x2(p[0], p[1]);
-    dS[i / 2] = pack_bf16x2(g[0], g[1]);
-  }
-}
-
-// D accumulator columns of this thread's row from TMEM, times `mul`, to a global fp32
-// row (or zeros when the row got no work).
-template <int D>
-__device__ __forceinline__ void store_acc_row(uint32_t taddr, bool have, bool valid, float mul, float* dst) {
-#pragma unroll
-  for (int c = 0; c < D / 32; ++c) {
-    uint32_t r[32];
-    if (have) {
-      tmem_ld32(taddr + c * 32, r);
-      tmem_ld_wait(r);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) r[i] = 0u;
-    }
-    if (valid) {
-      float4* out = reinterpret_cast<float4*>(dst + c * 32);
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        out[i] = make_float4(__uint_as_float(r[4 * i]) * mul, __uint_as_float(r[4 * i + 1]) * mul,
-                             __uint_as_float(r[4 * i + 2]) * mul, __uint_as_float(r[4 * i + 3]) * mul);
-    }
-  }
-}
 
 // Columns [C0, C0 + NC) of this thread's fp32 accumulator row r (times mul), written to
 // the calling warp's rows of a staging area in the layout of TMA's 128-byte swizzled fp32
@@ -163,18 +125,40 @@ __device__ __forceinline__ void store_acc_tma(uint32_t stage, int r, uint32_t ta
       tma_store_3d(map, stage + (uint32_t)((c - C0 / 32) * (128 * 128) + quad * 32 * 128), c * 32, row0 + quad * 32,
                    plane);
     bulk_commit();
-    bulk_wait_all();  // the CTA exits next: the stores must have read shared memory
+    bulk_wait_all();  // the staging area is reused or the CTA exits next
   }
   __syncwarp();
 }
 
+// dQ_step(128 x D) = dS K: A = dS^T in shared memory read MN-major (query columns in
+// 64-element blocks 16 KB apart), B = the K tile read MN-major (d columns in 64-element
+// blocks 16 KB apart); k-step kk covers keys 16 kk .. 16 kk + 15, 16 rows of 128 bytes.
+template <int D>
+__device__ __forceinline__ void issue_ds_k(uint32_t d_tmem, Desc ds, Desc k) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 1, 1);
+#pragma unroll
+  for (int kk = 0; kk < 128 / 16; ++kk) {
+    const uint32_t off = (uint32_t)((kk * 16 * 128) >> 4);
+    mma_ss_w(d_tmem, ds.lo + off, ds.hi, k.lo + off, k.hi, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
 struct BwdBars {
-  uint64_t fixed_full;  // the CTA's own tiles (K and V, or Q and dO) have landed
-  uint64_t stage_full[2];
-  uint64_t stage_empty[2];
-  uint64_t s_full[2];   // half h of the step's two score-like products is in TMEM
-  uint64_t p_full[2];   // P and/or dS of half h written back (4 warps)
-  uint64_t o_final;     // the last accumulation is done
+  uint64_t fixed_full;   // K and V of the CTA's key tile have landed
+  uint64_t q_full[2];    // Q of a step has landed (two-stage ring)
+  uint64_t q_empty[2];   // S and dK of the step are done with it
+  uint64_t do_full;      // dO of the step has landed (one stage)
+  uint64_t do_empty;     // dP and dV of the step are done with it
+  uint64_t s_full;       // S^T of the step is in TMEM
+  uint64_t dp_full;      // dP^T of the step is in TMEM
+  uint64_t p_full[2];    // P^T of query half h written over S^T (4 warps each)
+  uint64_t ds_full[2];   // dS^T of query half h written over dP^T and to shared memory (4 warps each)
+  uint64_t ds_free;      // dQ of the step is done with the shared dS^T
+  uint64_t dq_full;      // dQ_step is in TMEM
+  uint64_t dq_empty;     // the drain has read dQ_step out of TMEM (4 warps)
+  uint64_t stat_full;    // LSE and Delta of the step staged
+  uint64_t stat_free;    // the elementwise warps are done with them (8 warps)
+  uint64_t o_final;      // the last dK / dV accumulation is done
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -182,41 +166,31 @@ struct BwdBars {
 
 template <int D>
 struct BwdCfg {
-  // warp 0 TMA, 1 MMA, 2-3 statistics (dK/dV kernel), 4-7 and 8-11 the elementwise pass
-  // of query (dK/dV) or key (dQ) half 0 and half 1 of each step
-  static constexpr int THREADS = 384;
-  static constexpr int T = 128;  // rows of every tile
-  static constexpr int TILE_BYTES = T * D * 2;
-  static constexpr int OFF_FIXED = 0;                       // two tiles
-  static constexpr int OFF_RING = 2 * TILE_BYTES;           // 2 stages x two tiles
-  static constexpr int OFF_STAT = OFF_RING + 4 * TILE_BYTES;  // dK/dV kernel: [stage][L2 | delta][128]
-  static constexpr int OFF_BAR = OFF_STAT + 2 * 2 * 128 * 4;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + 1 KB alignment slack
+  // warp 0 loads K, V and Q, warp 1 issues the MMAs, warp 2 stages the statistics, warp 3
+  // loads dO; warps 4-7 and 8-11 run the elementwise pass of query columns 0-63 and
+  // 64-127 of each step; warps 12-15 drain dQ_step to global memory
+  static constexpr int THREADS = 512;
+  static constexpr int TILE_BYTES = 128 * D * 2;               // one bf16 tile of 128 rows
+  static constexpr int OFF_FIXED = 0;                          // K, V
+  static constexpr int OFF_Q = 2 * TILE_BYTES;                 // 2 stages of Q
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE_BYTES;        // 1 stage of dO
+  static constexpr int OFF_DS = OFF_DO + TILE_BYTES;           // dS^T: 128 keys x 128 queries, bf16
+  static constexpr int OFF_STG = OFF_DS + 128 * 128 * 2;       // dQ staging: 64 columns x 128 rows, fp32
+  static constexpr int OFF_STAT = OFF_STG + 2 * 128 * 128;     // L2 [128] | Delta [128] of the step
+  static constexpr int OFF_BAR = OFF_STAT + 2 * 128 * 4;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;            // + 1 KB alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
-  // S and dP in two 64-column halves each (half h at +64h), then the accumulators
-  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC0 = 256, COL_ACC1 = 256 + D;
+  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
+  static constexpr uint32_t COL_DQ = D == 128 ? COL_DP : 256 + 2 * D;
   static constexpr int HALF_ROWS_BYTES = 64 * 128;  // offset of rows 64.. inside a 64-column chunk
+  // registers per thread after the split (launch: 128 x 512 threads): warps 0-3 need few,
+  // the elementwise warps hold P for the step, the drain warps hold dQ_step's row
+  static constexpr int REGS_CTRL = 88, REGS_EW = 144, REGS_DRAIN = 136;
+  static_assert(REGS_CTRL + 2 * REGS_EW + REGS_DRAIN == 4 * 128, "register split must add up to the launch's");
+  static_assert(sizeof(BwdBars) <= 256, "barrier block");
 };
 
-__device__ __forceinline__ void bwd_init_bars(BwdBars* bars, int stage_full_count) {
-  mbar_init(&bars->fixed_full, 1);
-  for (int s = 0; s < 2; ++s) {
-    mbar_init(&bars->stage_full[s], stage_full_count);
-    mbar_init(&bars->stage_empty[s], 1);
-  }
-  for (int h = 0; h < 2; ++h) {
-    mbar_init(&bars->s_full[h], 1);
-    mbar_init(&bars->p_full[h], 4);
-  }
-  mbar_init(&bars->o_final, 1);
-  mbar_init(&bars->drain, 1);
-  bars->abort_flag = 0;
-  fence_mbar_init();
-}
-
-// ----------------------------------------------------------------------- dK / dV
-
-// Steps of a dK/dV CTA: (query head of the group, q-tile), q-tiles from qt_lo on.
+// Steps of a CTA: (query head of the group, q-tile), q-tiles from qt_lo on.
 __device__ __forceinline__ int kv_qt_lo(const BwdArgs& a, int kt) {
   if (!a.causal) return 0;
   const long long x = (long long)kt * 128 - (a.Nk - a.Nq);  // earliest query that sees key kt*128
@@ -226,7 +200,7 @@ __device__ __forceinline__ int kv_qt_lo(const BwdArgs& a, int kt) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(384, 1) attn_bwd_dkdv_kernel(const __grid_constant__ BwdArgs a) {
+__global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant__ BwdArgs a) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -245,10 +219,31 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkdv_kernel(const __grid_cons
   const int qt_lo = kv_qt_lo(a, kt);
   const int nqt = a.n_qtiles - qt_lo;
   const int nsteps = a.group * nqt;
-  auto step_bh = [&](int j) { return (size_t)b * a.Hq + (size_t)kvh * a.group + j / nqt; };
+  auto step_bh = [&](int j) { return b * a.Hq + kvh * a.group + j / nqt; };
   auto step_q0 = [&](int j) { return (qt_lo + j % nqt) * 128; };
 
-  if (threadIdx.x == 0) bwd_init_bars(bars, 3);  // TMA + the two stats warps
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->fixed_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->q_full[s], 1);
+      mbar_init(&bars->q_empty[s], 1);
+      mbar_init(&bars->p_full[s], 4);
+      mbar_init(&bars->ds_full[s], 4);
+    }
+    mbar_init(&bars->do_full, 1);
+    mbar_init(&bars->do_empty, 1);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->dp_full, 1);
+    mbar_init(&bars->ds_free, 1);
+    mbar_init(&bars->dq_full, 1);
+    mbar_init(&bars->dq_empty, 4);
+    mbar_init(&bars->stat_full, 1);
+    mbar_init(&bars->stat_free, 8);
+    mbar_init(&bars->o_final, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
@@ -258,162 +253,260 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkdv_kernel(const __grid_cons
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const uint32_t sK = smem_u32(smem + C::OFF_FIXED), sV = sK + C::TILE_BYTES;
-  const uint32_t sRing = smem_u32(smem + C::OFF_RING);
+  const uint32_t sQ0 = smem_u32(smem + C::OFF_Q), sDO = smem_u32(smem + C::OFF_DO);
+  const uint32_t sDS = smem_u32(smem + C::OFF_DS), sSTG = smem_u32(smem + C::OFF_STG);
+  auto q_stage = [&](int j) { return sQ0 + (uint32_t)((j & 1) * C::TILE_BYTES); };
 
-  if (warp == 0) {
-    // ================= TMA: K and V of the tile once, then Q and dO of every step
-    if (lane == 0) {
-      tma_prefetch_map(&a.tm_q);
-      tma_prefetch_map(&a.tm_do);
-      mbar_arrive_expect_tx(&bars->fixed_full, 2 * C::TILE_BYTES);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(smem + C::OFF_FIXED + c * (128 * 128), &a.tm_k, &bars->fixed_full, c * 64, k0, bkv);
-        tma_load_3d(smem + C::OFF_FIXED + C::TILE_BYTES + c * (128 * 128), &a.tm_v, &bars->fixed_full, c * 64, k0,
-                    bkv);
-      }
-      int j = 0;
-      for (; j < nsteps; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait(&bars->stage_empty[st], ((j >> 1) - 1) & 1, abort_flag, a.timeout_ns)) break;
-        mbar_arrive_expect_tx(&bars->stage_full[st], 2 * C::TILE_BYTES);
-        uint8_t* dst = smem + C::OFF_RING + st * 2 * C::TILE_BYTES;
+  if (warp < 4) {
+    setmaxnreg_dec<C::REGS_CTRL>();
+    if (warp == 0) {
+      // ================= TMA: K and V of the tile once, then Q of every step
+      if (lane == 0 && nsteps > 0) {
+        tma_prefetch_map(&a.tm_q);
+        mbar_arrive_expect_tx(&bars->fixed_full, 2 * C::TILE_BYTES);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(dst + c * (128 * 128), &a.tm_q, &bars->stage_full[st], c * 64, step_q0(j), (int)step_bh(j));
-          tma_load_3d(dst + C::TILE_BYTES + c * (128 * 128), &a.tm_do, &bars->stage_full[st], c * 64, step_q0(j),
-                      (int)step_bh(j));
+          tma_load_3d(smem + C::OFF_FIXED + c * (128 * 128), &a.tm_k, &bars->fixed_full, c * 64, k0, bkv);
+          tma_load_3d(smem + C::OFF_FIXED + C::TILE_BYTES + c * (128 * 128), &a.tm_v, &bars->fixed_full, c * 64, k0,
+                      bkv);
         }
-      }
-      // drain: the copies in flight must land before the CTA exits
-      mbar_wait(&bars->fixed_full, 0, abort_flag, a.timeout_ns, false);
-      for (int st = 0; st < 2 && st < j; ++st) {
-        const int last = j - 1 - ((j - 1 - st) & 1);  // last step that used stage st
-        mbar_wait(&bars->stage_full[st], (last >> 1) & 1, abort_flag, a.timeout_ns, false);
-      }
-    }
-  } else if (warp == 2 || warp == 3) {
-    // ================= per step: L2 (log-sum-exp in log2 units) and Delta of its 128 queries
-    const int t = threadIdx.x - 64;  // 0..63
-    for (int j = 0; j < nsteps; ++j) {
-      const int st = j & 1;
-      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars->stage_empty[st], ((j >> 1) - 1) & 1, abort_flag,
-                                                       a.timeout_ns)))
-        break;
-      const size_t bh = step_bh(j);
-      const int q0 = step_q0(j);
-      float* L2 = stat + st * 256;
+        int j = 0;
+        for (; j < nsteps; ++j) {
+          const int st = j & 1;
+          if (j >= 2 && !mbar_wait(&bars->q_empty[st], ((j >> 1) - 1) & 1, abort_flag, a.timeout_ns)) break;
+          mbar_arrive_expect_tx(&bars->q_full[st], C::TILE_BYTES);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int c = t + 64 * h;
-        const int q = q0 + c;
-        L2[c] = lse2_of(a, bh, q);
-        L2[128 + c] = (q < a.Nq) ? __ldg(&a.delta[bh * a.Nq + q]) : 0.f;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->stage_full[st]);
-    }
-  } else if (warp == 1) {
-    // ================= MMA issuer (whole warp, one elected lane issues)
-    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.timeout_ns));
-    };
-    if (nsteps > 0) {
-      const Desc dk = desc_sw128(sK, 16, 1024), dvk = desc_sw128(sV, 16, 1024);
-      // Each step is split in two halves of 64 queries, so that the softmax warps work on
-      // one half while the tensor core computes the other:
-      //   S^T_h = K Q_h^T, dP^T_h = V dO_h^T  (64 columns each), then after p_full[h]
-      //   dV += P^T_h dO_h, dK += dS^T_h Q_h  (contraction over the half's 64 queries).
-      // The next step's half h overwrites P_h / dS_h only after those products were
-      // issued (this thread issues in order).
-      auto stage_q = [&](int j) { return sRing + (j & 1) * 2 * C::TILE_BYTES; };
-      auto issue_s = [&](int j, int h) {
-        const uint32_t sQ = stage_q(j) + h * C::HALF_ROWS_BYTES, sDO = sQ + C::TILE_BYTES;
-        if (elect_one()) {
-          tc_fence_after();
-          issue_qk_rows<D, 64>(tmem + C::COL_S + 64 * h, dk, desc_sw128(sQ, 16, 1024));
-          issue_qk_rows<D, 64>(tmem + C::COL_DP + 64 * h, dvk, desc_sw128(sDO, 16, 1024));
-          tc_commit(&bars->s_full[h]);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem + C::OFF_Q + st * C::TILE_BYTES + c * (128 * 128), &a.tm_q, &bars->q_full[st], c * 64,
+                        step_q0(j), step_bh(j));
         }
-        __syncwarp();
+        // drain: the copies in flight must land before the CTA exits
+        mbar_wait(&bars->fixed_full, 0, abort_flag, a.timeout_ns, false);
+        for (int st = 0; st < 2 && st < j; ++st) {
+          const int last = j - 1 - ((j - 1 - st) & 1);  // last step that used stage st
+          mbar_wait(&bars->q_full[st], (last >> 1) & 1, abort_flag, a.timeout_ns, false);
+        }
+      }
+    } else if (warp == 3) {
+      // ================= TMA: dO of every step into its single stage
+      if (lane == 0 && nsteps > 0) {
+        tma_prefetch_map(&a.tm_do);
+        int j = 0;
+        for (; j < nsteps; ++j) {
+          if (j >= 1 && !mbar_wait(&bars->do_empty, (j - 1) & 1, abort_flag, a.timeout_ns)) break;
+          mbar_arrive_expect_tx(&bars->do_full, C::TILE_BYTES);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem + C::OFF_DO + c * (128 * 128), &a.tm_do, &bars->do_full, c * 64, step_q0(j),
+                        step_bh(j));
+        }
+        if (j > 0) mbar_wait(&bars->do_full, (j - 1) & 1, abort_flag, a.timeout_ns, false);
+      }
+    } else if (warp == 1) {
+      // ================= MMA issuer (whole warp, one elected lane issues).  Per step j:
+      //   dV += P^T dO, S^T(j+1), dK += dS^T Q, dQ_step = dS K, dP^T(j+1)
+      // so that the next step's scores are computed while the elementwise warps work.
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.timeout_ns));
       };
-      auto issue_acc = [&](int j, int h) {
-        const uint32_t sQ = stage_q(j) + h * C::HALF_ROWS_BYTES, sDO = sQ + C::TILE_BYTES;
-        const bool acc = j > 0 || h > 0;
-        if (elect_one()) {
-          tc_fence_after();
-          issue_pv_ts_w<D, 64>(tmem + C::COL_ACC1, tmem + C::COL_S + 64 * h, desc_sw128(sDO, 128 * 128, 1024), acc);
-          issue_pv_ts_w<D, 64>(tmem + C::COL_ACC0, tmem + C::COL_DP + 64 * h, desc_sw128(sQ, 128 * 128, 1024), acc);
+      if (nsteps > 0) {
+        const Desc dk = desc_sw128(sK, 16, 1024), dv = desc_sw128(sV, 16, 1024);
+        const Desc ddo = desc_sw128(sDO, 16, 1024);
+        auto issue_s = [&](int j) {  // S^T = K Q^T
+          if (elect_one()) {
+            tc_fence_after();
+            issue_qk_rows<D, 128>(tmem + C::COL_S, dk, desc_sw128(q_stage(j), 16, 1024));
+            tc_commit(&bars->s_full);
+          }
+          __syncwarp();
+        };
+        auto issue_dp = [&]() {  // dP^T = V dO^T
+          if (elect_one()) {
+            tc_fence_after();
+            issue_qk_rows<D, 128>(tmem + C::COL_DP, dv, ddo);
+            tc_commit(&bars->dp_full);
+          }
+          __syncwarp();
+        };
+        bool ok = wait_all(&bars->fixed_full, 0) && wait_all(&bars->q_full[0], 0);
+        if (ok) issue_s(0);
+        ok = ok && wait_all(&bars->do_full, 0);
+        if (ok) issue_dp();
+        for (int j = 0; j < nsteps && ok; ++j) {
+          const bool more = j + 1 < nsteps;
+          const uint32_t sQ = q_stage(j);
+          // dV += P^T dO, one query half at a time (A = P^T half h from TMEM)
+          for (int h = 0; h < 2 && ok; ++h) {
+            ok = wait_all(&bars->p_full[h], j & 1);
+            if (ok && elect_one()) {
+              tc_fence_after();
+              issue_pv_ts_w<D, 64>(tmem + C::COL_DV, tmem + C::COL_S + 64 * h,
+                                   desc_sw128(sDO + h * C::HALF_ROWS_BYTES, 128 * 128, 1024), j > 0 || h > 0);
+            }
+            __syncwarp();
+          }
+          if (!ok) break;
+          if (elect_one()) tc_commit(&bars->do_empty);  // dP and dV are done with dO
+          __syncwarp();
+          // the S columns are free once dV has been issued (products run in issue order)
+          if (more) {
+            if (!wait_all(&bars->q_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) break;
+            issue_s(j + 1);
+          }
+          // dK += dS^T Q, one query half at a time (A = dS^T half h from TMEM)
+          for (int h = 0; h < 2 && ok; ++h) {
+            ok = wait_all(&bars->ds_full[h], j & 1);
+            if (ok && elect_one()) {
+              tc_fence_after();
+              issue_pv_ts_w<D, 64>(tmem + C::COL_DK, tmem + C::COL_DP + 64 * h,
+                                   desc_sw128(sQ + h * C::HALF_ROWS_BYTES, 128 * 128, 1024), j > 0 || h > 0);
+            }
+            __syncwarp();
+          }
+          if (!ok) break;
+          if (elect_one()) tc_commit(&bars->q_empty[j & 1]);  // S and dK are done with Q
+          __syncwarp();
+          // dQ_step = dS K; at d = 64 it has its own columns, which the drain must have
+          // emptied of the previous step's
+          if (D == 64 && j > 0 && !wait_all(&bars->dq_empty, (j - 1) & 1)) break;
+          if (elect_one()) {
+            tc_fence_after();
+            issue_ds_k<D>(tmem + C::COL_DQ, desc_sw128(sDS, 128 * 128, 1024), desc_sw128(sK, 128 * 128, 1024));
+            tc_commit(&bars->ds_free);
+            tc_commit(&bars->dq_full);
+            if (!more) tc_commit(&bars->o_final);
+          }
+          __syncwarp();
+          if (more) {
+            // at d = 128 dP^T of the next step goes where dQ_step is: wait for the drain
+            if (D == 128 && !wait_all(&bars->dq_empty, j & 1)) break;
+            if (!wait_all(&bars->do_full, (j + 1) & 1)) break;
+            issue_dp();
+          }
+        }
+        if (elect_one()) tc_commit(&bars->drain);
+        __syncwarp();
+        mbar_wait(&bars->drain, 0, abort_flag, a.timeout_ns, false);
+      }
+    } else {
+      // ================= warp 2: LSE (log2 units) and Delta of each step's 128 queries
+      for (int j = 0; j < nsteps; ++j) {
+        const size_t bh = step_bh(j);
+        const int q0 = step_q0(j);
+        float l[4], d[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int q = q0 + lane + 32 * i;
+          l[i] = lse2_of(a, bh, q);
+          d[i] = (q < a.Nq) ? __ldg(&a.delta[bh * a.Nq + q]) : 0.f;
+        }
+        if (j >= 1 &&
+            !__all_sync(0xffffffffu, mbar_wait(&bars->stat_free, (j - 1) & 1, abort_flag, a.timeout_ns)))
+          break;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          stat[lane + 32 * i] = l[i];
+          stat[128 + lane + 32 * i] = d[i];
         }
         __syncwarp();
-      };
-      bool ok = wait_all(&bars->fixed_full, 0) && wait_all(&bars->stage_full[0], 0);
-      if (ok) {
-        issue_s(0, 0);
-        issue_s(0, 1);
+        if (lane == 0) mbar_arrive(&bars->stat_full);
       }
-      for (int j = 0; j < nsteps && ok; ++j) {
-        const bool more = j + 1 < nsteps;
-        if (!wait_all(&bars->p_full[0], j & 1)) break;
-        issue_acc(j, 0);
-        if (more) {
-          if (!wait_all(&bars->stage_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) break;
-          issue_s(j + 1, 0);
-        }
-        if (!wait_all(&bars->p_full[1], j & 1)) break;
-        issue_acc(j, 1);
-        if (elect_one()) {
-          tc_commit(&bars->stage_empty[j & 1]);  // Q, dO and the statistics of step j
-          if (!more) tc_commit(&bars->o_final);
-        }
-        __syncwarp();
-        if (more) issue_s(j + 1, 1);
-      }
-      if (elect_one()) tc_commit(&bars->drain);
-      __syncwarp();
-      mbar_wait(&bars->drain, 0, abort_flag, a.timeout_ns, false);
     }
-  } else {
-    // ================= warps 4-7 (half 0) and 8-11 (half 1): one key row per thread, the
-    // half's 64 query columns of every step
+  } else if (warp < 12) {
+    setmaxnreg_inc<C::REGS_EW>();
+    // ================= warps 4-7 (query half 0) and 8-11 (half 1): one key row per
+    // thread, the half's 64 query columns of every step
     const int h = warp >= 8 ? 1 : 0;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int k = k0 + r;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::COL_S, tDP = tmem + lane_off + C::COL_DP;
+    const uint32_t tS = tmem + lane_off + C::COL_S + 64 * h, tDP = tmem + lane_off + C::COL_DP + 64 * h;
+    const uint32_t ds_row = sDS + (uint32_t)(h * (128 * 128) + r * 128);
     const int off = a.Nk - a.Nq;
     bool ok = true;
     for (int j = 0; j < nsteps && ok; ++j) {
-      const int st = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->stage_full[st], (j >> 1) & 1, abort_flag, a.timeout_ns))) {
+      const int q0 = step_q0(j);
+      // first visible query column of this key row: q >= k - off under the causal mask;
+      // none for a key past the sequence (its K row is zero-filled, its P must be 0)
+      const int lo = (k >= a.Nk ? (1 << 20) : (a.causal ? k - off - q0 : 0)) - 64 * h;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->stat_full, j & 1, abort_flag, a.timeout_ns) &&
+                                       mbar_wait(&bars->s_full, j & 1, abort_flag, a.timeout_ns))) {
         ok = false;
         break;
       }
-      const float* L2 = stat + st * 256;
-      // visible query columns of this key row: q >= k - off (causal)
-      const int lo = a.causal ? k - off - step_q0(j) : -1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[h], j & 1, abort_flag, a.timeout_ns))) {
+      tc_fence_after();
+      // ---- P^T = 2^(s scale log2e - L2) over the visible columns; p keeps it in fp32
+      uint32_t p[2][32];
+      tmem_ld32(tS, p[0]);
+      tmem_ld32(tS + 32, p[1]);
+      tmem_ld_wait(p[0]);
+      tmem_ld_wait(p[1]);
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const float4* L2 = reinterpret_cast<const float4*>(stat + 64 * h + 32 * cc);
+        uint32_t P[16];
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 l = L2[i4];
+          const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 4 * i4 + e;
+            const float y = fmaf(__uint_as_float(p[cc][i]), a.scale_log2, -lv[e]);
+            p[cc][i] = __float_as_uint((32 * cc + i >= lo) ? ex2(y) : 0.f);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          P[i] = pack_bf16x2(__uint_as_float(p[cc][2 * i]), __uint_as_float(p[cc][2 * i + 1]));
+        tmem_st16(tS + 16 * cc, P);  // over the half's columns already read
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full[h]);
+      // ---- dS^T = P^T o (dP^T - Delta): bf16 over dP^T (for dK) and to shared memory
+      // in the 128-byte swizzled layout (for dQ)
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&bars->dp_full, j & 1, abort_flag, a.timeout_ns) &&
+                          (j == 0 || mbar_wait(&bars->ds_free, (j - 1) & 1, abort_flag, a.timeout_ns)))) {
         ok = false;
         break;
       }
       tc_fence_after();
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        const int c0 = 64 * h + 32 * cc;  // first query column of the chunk
-        uint32_t sv[32], dp[32], P[16], dS[16];
-        tmem_ld32(tS + c0, sv);
-        tmem_ld32(tDP + c0, dp);
-        tmem_ld_wait(sv);
+        uint32_t dp[32];
+        tmem_ld32(tDP + 32 * cc, dp);
         tmem_ld_wait(dp);
-        bwd_chunk(sv, dp, a.scale_log2, L2 + c0, L2 + 128 + c0, lo - c0, 31, P, dS);
-        tmem_st16(tS + 64 * h + 16 * cc, P);  // packed over the half's columns already read
-        tmem_st16(tDP + 64 * h + 16 * cc, dS);
+        const float4* Dl = reinterpret_cast<const float4*>(stat + 128 + 64 * h + 32 * cc);
+        uint32_t dS[16];
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 dl = Dl[i4];
+          const int i = 4 * i4;
+          dS[2 * i4] = pack_bf16x2(__uint_as_float(p[cc][i]) * (__uint_as_float(dp[i]) - dl.x),
+                                   __uint_as_float(p[cc][i + 1]) * (__uint_as_float(dp[i + 1]) - dl.y));
+          dS[2 * i4 + 1] = pack_bf16x2(__uint_as_float(p[cc][i + 2]) * (__uint_as_float(dp[i + 2]) - dl.z),
+                                       __uint_as_float(p[cc][i + 3]) * (__uint_as_float(dp[i + 3]) - dl.w));
+        }
+        tmem_st16(tDP + 16 * cc, dS);  // over the half's columns already read
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int gg = 4 * cc + g;  // 16-byte granule of the 128-byte row
+          st_shared_v4(ds_row + (uint32_t)((gg ^ (r & 7)) << 4), dS[4 * g], dS[4 * g + 1], dS[4 * g + 2],
+                       dS[4 * g + 3]);
+        }
       }
+      fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[h]);
+      if (lane == 0) {
+        mbar_arrive(&bars->ds_full[h]);
+        mbar_arrive(&bars->stat_free);
+      }
     }
     ok = __all_sync(0xffffffffu, ok);
     const bool have = nsteps > 0;
@@ -421,199 +514,65 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkdv_kernel(const __grid_cons
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_final, 0, abort_flag, a.timeout_ns));
       tc_fence_after();
     }
-    if (ok) {  // half 0's warps write dK, half 1's dV, each staged in one ring stage (free now)
-      const uint32_t stage = sRing + (uint32_t)(h * 2 * C::TILE_BYTES);
+    if (ok) {
+      // dK (half 0's warps) staged in the K/V tiles, dV (half 1's) in the Q stages; both
+      // are free once the last products are done
       if (h == 0)
-        store_acc_tma<0, D>(stage, r, tmem + lane_off + C::COL_ACC0, have, a.scale, &a.tm_dk, k0, a.Nk, bkv);
+        store_acc_tma<0, D>(sK, r, tmem + lane_off + C::COL_DK, have, a.scale, &a.tm_dk, k0, a.Nk, bkv);
       else
-        store_acc_tma<0, D>(stage, r, tmem + lane_off + C::COL_ACC1, have, 1.0f, &a.tm_dv, k0, a.Nk, bkv);
+        store_acc_tma<0, D>(sQ0, r, tmem + lane_off + C::COL_DV, have, 1.0f, &a.tm_dv, k0, a.Nk, bkv);
     }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
-  }
-}
-
-// ---------------------------------------------------------------------------- dQ
-
-template <int D>
-__global__ void __launch_bounds__(384, 1) attn_bwd_dq_kernel(const __grid_constant__ BwdArgs a) {
-  using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + C::OFF_BAR);
-  volatile int* abort_flag = &bars->abort_flag;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  // causal: the last q-tiles see the most K/V tiles, so they go first
-  const int qt = a.n_qtiles - 1 - (int)(blockIdx.x / (a.B * a.Hq));
-  const int bh = blockIdx.x % (a.B * a.Hq);  // b * Hq + hq
-  const int b = bh / a.Hq, hq = bh % a.Hq;
-  const int bkv = b * a.Hkv + hq / a.group;
-  const int q0 = qt * 128;
-  const int off = a.Nk - a.Nq;
-  int nsteps = a.n_ktiles;  // K/V tiles 0 .. nsteps-1
-  if (a.causal) {
-    const long long last = (long long)q0 + 127 + off;  // last key the tile's last row sees
-    const long long n = last < 0 ? 0 : last / 128 + 1;
-    nsteps = n < a.n_ktiles ? (int)n : a.n_ktiles;
-  }
-
-  if (threadIdx.x == 0) bwd_init_bars(bars, 1);
-  if (warp == 1) {
-    tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = bars->tmem_base;
-  const uint32_t sQ = smem_u32(smem + C::OFF_FIXED), sDO = sQ + C::TILE_BYTES;
-  const uint32_t sRing = smem_u32(smem + C::OFF_RING);
-
-  if (warp == 0) {
-    if (lane == 0 && nsteps > 0) {
-      tma_prefetch_map(&a.tm_k);
-      tma_prefetch_map(&a.tm_v);
-      mbar_arrive_expect_tx(&bars->fixed_full, 2 * C::TILE_BYTES);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(smem + C::OFF_FIXED + c * (128 * 128), &a.tm_q, &bars->fixed_full, c * 64, q0, bh);
-        tma_load_3d(smem + C::OFF_FIXED + C::TILE_BYTES + c * (128 * 128), &a.tm_do, &bars->fixed_full, c * 64, q0,
-                    bh);
-      }
-      int j = 0;
-      for (; j < nsteps; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait(&bars->stage_empty[st], ((j >> 1) - 1) & 1, abort_flag, a.timeout_ns)) break;
-        mbar_arrive_expect_tx(&bars->stage_full[st], 2 * C::TILE_BYTES);
-        uint8_t* dst = smem + C::OFF_RING + st * 2 * C::TILE_BYTES;
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(dst + c * (128 * 128), &a.tm_k, &bars->stage_full[st], c * 64, j * 128, bkv);
-          tma_load_3d(dst + C::TILE_BYTES + c * (128 * 128), &a.tm_v, &bars->stage_full[st], c * 64, j * 128, bkv);
-        }
-      }
-      mbar_wait(&bars->fixed_full, 0, abort_flag, a.timeout_ns, false);
-      for (int st = 0; st < 2 && st < j; ++st) {
-        const int last = j - 1 - ((j - 1 - st) & 1);
-        mbar_wait(&bars->stage_full[st], (last >> 1) & 1, abort_flag, a.timeout_ns, false);
-      }
-    }
-  } else if (warp == 1) {
-    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.timeout_ns));
-    };
-    if (nsteps > 0) {
-      const Desc dq = desc_sw128(sQ, 16, 1024), ddo = desc_sw128(sDO, 16, 1024);
-      // halves of 64 keys: S_h = Q K_h^T, dP_h = dO V_h^T, then dQ += dS_h K_h
-      auto stage_k = [&](int j) { return sRing + (j & 1) * 2 * C::TILE_BYTES; };
-      auto issue_s = [&](int j, int h) {
-        const uint32_t sK = stage_k(j) + h * C::HALF_ROWS_BYTES, sV = sK + C::TILE_BYTES;
-        if (elect_one()) {
-          tc_fence_after();
-          issue_qk_rows<D, 64>(tmem + C::COL_S + 64 * h, dq, desc_sw128(sK, 16, 1024));
-          issue_qk_rows<D, 64>(tmem + C::COL_DP + 64 * h, ddo, desc_sw128(sV, 16, 1024));
-          tc_commit(&bars->s_full[h]);
-        }
-        __syncwarp();
-      };
-      auto issue_acc = [&](int j, int h) {
-        const uint32_t sK = stage_k(j) + h * C::HALF_ROWS_BYTES;
-        if (elect_one()) {
-          tc_fence_after();
-          issue_pv_ts_w<D, 64>(tmem + C::COL_ACC0, tmem + C::COL_S + 64 * h, desc_sw128(sK, 128 * 128, 1024),
-                               j > 0 || h > 0);
-        }
-        __syncwarp();
-      };
-      bool ok = wait_all(&bars->fixed_full, 0) && wait_all(&bars->stage_full[0], 0);
-      if (ok) {
-        issue_s(0, 0);
-        issue_s(0, 1);
-      }
-      for (int j = 0; j < nsteps && ok; ++j) {
-        const bool more = j + 1 < nsteps;
-        if (!wait_all(&bars->p_full[0], j & 1)) break;
-        issue_acc(j, 0);
-        if (more) {
-          if (!wait_all(&bars->stage_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) break;
-          issue_s(j + 1, 0);
-        }
-        if (!wait_all(&bars->p_full[1], j & 1)) break;
-        issue_acc(j, 1);
-        if (elect_one()) {
-          tc_commit(&bars->stage_empty[j & 1]);
-          if (!more) tc_commit(&bars->o_final);
-        }
-        __syncwarp();
-        if (more) issue_s(j + 1, 1);
-      }
-      if (elect_one()) tc_commit(&bars->drain);
-      __syncwarp();
-      mbar_wait(&bars->drain, 0, abort_flag, a.timeout_ns, false);
-    }
-  } else if (warp >= 4) {
-    // ================= warps 4-7 (half 0) and 8-11 (half 1): one query row per thread,
-    // the half's 64 key columns of every step
-    const int h = warp >= 8 ? 1 : 0;
+  } else {
+    setmaxnreg_inc<C::REGS_DRAIN>();
+    // ================= warps 12-15: dQ_step out of TMEM (one query row per thread) into
+    // registers, which frees its columns at once; then, 64 columns at a time, times scale
+    // into the staging buffer and added to dQ by TMA reduce-adds that run in the
+    // background of the next steps
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const int q = q0 + r;
-    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::COL_S, tDP = tmem + lane_off + C::COL_DP;
-    const float L2 = lse2_of(a, (size_t)bh, q);
-    const float dl = (q < a.Nq) ? __ldg(&a.delta[(size_t)bh * a.Nq + q]) : 0.f;
-    float L2v[32], dlv[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      L2v[i] = L2;
-      dlv[i] = dl;
-    }
-    bool ok = true;
-    for (int j = 0; j < nsteps && ok; ++j) {
-      // visible key columns of this query row: key < Nk, and key <= q + off (causal)
-      int hi = a.Nk - 1 - j * 128;
-      if (a.causal) hi = min(hi, q + off - j * 128);
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[h], j & 1, abort_flag, a.timeout_ns))) {
-        ok = false;
-        break;
-      }
+    const uint32_t tQ = tmem + ((uint32_t)(quad * 32) << 16) + C::COL_DQ;
+    const uint32_t stg_rows = sSTG + (uint32_t)(r * 128);
+    for (int j = 0; j < nsteps; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->dq_full, j & 1, abort_flag, a.timeout_ns))) break;
       tc_fence_after();
+      uint32_t v[D / 32][32];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c0 = 64 * h + 32 * cc;
-        uint32_t sv[32], dp[32], P[16], dS[16];
-        tmem_ld32(tS + c0, sv);
-        tmem_ld32(tDP + c0, dp);
-        tmem_ld_wait(sv);
-        tmem_ld_wait(dp);
-        bwd_chunk(sv, dp, a.scale_log2, L2v, dlv, 0, hi - c0, P, dS);
-        tmem_st16(tS + 64 * h + 16 * cc, dS);  // over the half's S columns already read
-      }
-      tmem_st_wait();
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(tQ + c * 32, v[c]);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_ld_wait(v[c]);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[h]);
+      if (lane == 0) mbar_arrive(&bars->dq_empty);
+      const int q0 = step_q0(j);
+      const bool rows_in = q0 + quad * 32 < a.Nq;
+#pragma unroll
+      for (int half = 0; half < D / 64; ++half) {
+        // the previous reduce-adds must have read the staging rows of this warp
+        if (lane == 0) bulk_wait_read();
+        __syncwarp();
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const uint32_t* w = v[2 * half + cc];
+          const uint32_t row = stg_rows + (uint32_t)(cc * (128 * 128));
+#pragma unroll
+          for (int g = 0; g < 8; ++g)
+            st_shared_v4(row + (uint32_t)((g ^ (r & 7)) << 4), __float_as_uint(__uint_as_float(w[4 * g]) * a.scale),
+                         __float_as_uint(__uint_as_float(w[4 * g + 1]) * a.scale),
+                         __float_as_uint(__uint_as_float(w[4 * g + 2]) * a.scale),
+                         __float_as_uint(__uint_as_float(w[4 * g + 3]) * a.scale));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && rows_in) {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc)
+            tma_reduce_add_3d(&a.tm_dq, sSTG + (uint32_t)(cc * (128 * 128) + quad * 32 * 128), (2 * half + cc) * 32,
+                              q0 + quad * 32, step_bh(j));
+          bulk_commit();
+        }
+      }
     }
-    ok = __all_sync(0xffffffffu, ok);
-    const bool have = nsteps > 0;
-    if (ok && have) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_final, 0, abort_flag, a.timeout_ns));
-      tc_fence_after();
-    }
-    if (ok) {  // each half's warps write half of the row's columns, staged in the (free) ring
-      const uint32_t stage = sRing + (uint32_t)(h * (D / 64) * (128 * 128));
-      if (h == 0)
-        store_acc_tma<0, D / 2>(stage, r, tmem + lane_off + C::COL_ACC0, have, a.scale, &a.tm_dq, q0, a.Nq, bh);
-      else
-        store_acc_tma<D / 2, D / 2>(stage, r, tmem + lane_off + C::COL_ACC0, have, a.scale, &a.tm_dq, q0, a.Nq, bh);
-    }
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();

@@ -457,9 +457,9 @@ def timed_launches(step, K, W, flush, stream, dist, dev):
 
 
 def bwd_record(args, ab, name, dev, stream, dist, peaks, peak_src, K, W, cpu=True):
-    """Backward pass (attn_bwd: delta, dK/dV and dQ kernels) of a prefill workload.  FLOPs are
-    the method's five products, 2.5x the forward's (causal halved), as the pages' FA figures
-    count them; the dQ kernel's recomputation of S and dP is not counted."""
+    """Backward pass (attn_bwd: the delta kernel, then one pass that computes the five
+    products per block) of a prefill workload.  FLOPs are the method's five products, 2.5x
+    the forward's (causal halved), as the pages' FA figures count them."""
     shape = synth.WORKLOADS[name]
     seed = rank_seed(synth.workload_seed(name), dist.rank)
     pre = make_prefill(shape, seed, dev)
@@ -494,10 +494,10 @@ def bwd_record(args, ab, name, dev, stream, dist, peaks, peak_src, K, W, cpu=Tru
                      "traffic": profiled_traffic(f"attn_bwd_{name}.md") if name in ("gqa_causal_2k", "gqa_causal_16k")
                      else None,
                      "peak_source": f"{peak_src} bf16_tflops (burst cuBLAS)",
-                     "kernel": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel + attn_bwd_delta_kernel (one call)",
+                     "kernel": "attn_bwd_kernel + attn_bwd_delta_kernel (one call)",
                      "flops_per_launch": flops},
         "l2": "L2 flushed before every call by writing a 256 MB buffer",
-        "clocks": clk, "gpu_launches": 3 * K,
+        "clocks": clk, "gpu_launches": 2 * K,
     }
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline and cpu:
         rec["cpu_baseline"] = oracle_backward_sample(shape, pre["host"], do.cpu(), scale, flops, args.cpu_seconds / 2)

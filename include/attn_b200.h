@@ -186,7 +186,9 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Nq);
  *   k, v        device, bf16 [B, Hkv, Nk, d]
  *   o, lse      device, the forward's outputs: bf16 O [B, Hq, Nq, d] and fp32 natural
  *               log-sum-exp [B, Hq, Nq] (as written by attn_fwd on the same inputs)
- *   dq          device, fp32 [B, Hq, Nq, d]   (written)
+ *   dq          device, fp32 [B, Hq, Nq, d]   (written: cleared by the call, then
+ *               accumulated over the key tiles by additions in L2, so nothing else may
+ *               write it while the call runs)
  *   dk, dv      device, fp32 [B, Hkv, Nk, d]  (written; for grouped heads the sums over
  *               the Hq/Hkv query heads that share the K/V head)
  *   d           64 or 128 (256: ATTN_ERR_UNSUPPORTED);  causal as in attn_fwd.
@@ -194,10 +196,7 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Nq);
  *               16-byte aligned, owned by the caller (ATTN_ERR_WORKSPACE if too small).
  * Alignment: q, k, v, o, dout, dq, dk, dv 16-byte aligned.  A row with no visible key
  * (lse = -inf) gets zero gradient.  Nq = 0 writes dk = dv = 0; Nk = 0 writes dq = 0.
- * Streams: the call is ordered on `stream` like any other: its dQ kernel runs on a
- * library-owned stream that waits for the Delta pass enqueued on `stream`, and `stream`
- * waits for the dQ kernel before anything enqueued after the call (an event fork and
- * join, which CUDA graph capture records as such).
+ * Streams: both kernels of the call (Delta, then the gradients) run on `stream`.
  */
 attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                      const float* lse, float* dq, float* dk, float* dv, int B, int Hq, int Hkv,

@@ -1,7 +1,7 @@
 """The entry points inside a CUDA graph: a prefill, its backward pass and a paged decode
 step are captured once and replayed, and the replay must reproduce the eager calls bit
-for bit.  The backward pass forks its dQ kernel onto a second stream; the capture records
-that as a fork and a join."""
+for bit.  The backward pass accumulates dQ by additions in L2 whose order varies from run
+to run, so its dQ is compared within a few fp32 ulps of the eager call instead."""
 
 import math
 
@@ -43,7 +43,7 @@ def test_prefill_backward_decode_replay_matches_eager(cuda_device):
         ab.attn_bwd(q, k, v, o, do, lse, dq, dk, dv, True, scale, bws)
         ab.attn_decode_paged(dq_in, kp, vp, bt, sl, kv.page_size, do_, dlse, 1.0 / math.sqrt(d), dws)
 
-    # eager (also sets the kernels' shared-memory limits and creates the side stream)
+    # eager (also sets the kernels' shared-memory limits)
     step()
     torch.cuda.synchronize()
     assert ab.attn_get_device_status() == 0
@@ -58,7 +58,11 @@ def test_prefill_backward_decode_replay_matches_eager(cuda_device):
         g.replay()
     torch.cuda.synchronize()
     assert ab.attn_get_device_status() == 0
-    for ref, got in zip(eager, outs):
-        assert torch.equal(ref.view(torch.uint8), got.view(torch.uint8))
+    for i, (ref, got) in enumerate(zip(eager, outs)):
+        if got is dq:  # sums in L2 in an order that varies: a few fp32 roundings apart
+            assert torch.isfinite(got).all()
+            assert (got - ref).abs().max().item() <= 1e-5 * ref.abs().max().item()
+        else:
+            assert torch.equal(ref.view(torch.uint8), got.view(torch.uint8)), i
     del g
     assert np.isfinite(eager[0].float().cpu().numpy()).all()
