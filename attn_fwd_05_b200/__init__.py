@@ -19,6 +19,7 @@ from .binding import (  # noqa: F401
     attn_fwd_masked,
     attn_get_device_status,
     attn_quantize_fp8,
+    attn_debug_bwd_stall,
     attn_debug_decode_stall,
     attn_debug_exp2,
     attn_debug_fwd_stall,

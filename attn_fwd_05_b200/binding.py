@@ -47,6 +47,8 @@ SIGNATURES = {
     "attn_debug_exp2": (_I, [_P, _P, _I, _P]),
     "attn_debug_fwd_stall": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _I, _I,
                                   ctypes.c_uint64, _P]),
+    "attn_debug_bwd_stall": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I,
+                                  _P, ctypes.c_size_t, _I, _I, ctypes.c_uint64, _P]),
     "attn_debug_decode_stall": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P,
                                      ctypes.c_size_t, _I, _I, ctypes.c_uint64, _P]),
     "attn_get_device_status": (_I, [_P]),
@@ -208,11 +210,7 @@ def attn_bwd_workspace_size(B: int, Hq: int, Nq: int) -> int:
     return int(load_library().attn_bwd_workspace_size(B, Hq, Nq))
 
 
-def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, do: torch.Tensor,
-             lse: torch.Tensor, dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor, causal: bool, scale: float,
-             workspace: torch.Tensor | None = None, stream=None) -> None:
-    """Backward pass: fp32 dq [B, Hq, Nq, d], dk and dv [B, Hkv, Nk, d] from the bf16 inputs, the
-    forward's bf16 o and fp32 lse, and the bf16 upstream gradient do [B, Hq, Nq, d]."""
+def _bwd_args(q, k, v, o, do, lse, dq, dk, dv, causal, scale, workspace):
     lib = load_library()
     B, Hq, Nq, d = q.shape
     Hkv, Nk = k.shape[1], k.shape[2]
@@ -229,13 +227,21 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     need = lib.attn_bwd_workspace_size(B, Hq, Nq)
     if workspace is None:
         workspace = torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
-    st = lib.attn_bwd(_dev(q, "q", torch.bfloat16, 4), _dev(k, "k", torch.bfloat16, 4), _dev(v, "v", torch.bfloat16, 4),
-                      _dev(o, "o", torch.bfloat16, 4), _dev(do, "do", torch.bfloat16, 4),
-                      _dev(lse, "lse", torch.float32, 3), _dev(dq, "dq", torch.float32, 4),
-                      _dev(dk, "dk", torch.float32, 4), _dev(dv, "dv", torch.float32, 4),
-                      B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
-                      _dev(workspace, "workspace", torch.uint8, 1), workspace.numel(), _stream(stream))
-    _check(st, "attn_bwd")
+    return (_dev(q, "q", torch.bfloat16, 4), _dev(k, "k", torch.bfloat16, 4), _dev(v, "v", torch.bfloat16, 4),
+            _dev(o, "o", torch.bfloat16, 4), _dev(do, "do", torch.bfloat16, 4),
+            _dev(lse, "lse", torch.float32, 3), _dev(dq, "dq", torch.float32, 4),
+            _dev(dk, "dk", torch.float32, 4), _dev(dv, "dv", torch.float32, 4),
+            B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
+            _dev(workspace, "workspace", torch.uint8, 1), workspace.numel())
+
+
+def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, do: torch.Tensor,
+             lse: torch.Tensor, dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor, causal: bool, scale: float,
+             workspace: torch.Tensor | None = None, stream=None) -> None:
+    """Backward pass: fp32 dq [B, Hq, Nq, d], dk and dv [B, Hkv, Nk, d] from the bf16 inputs, the
+    forward's bf16 o and fp32 lse, and the bf16 upstream gradient do [B, Hq, Nq, d]."""
+    args = _bwd_args(q, k, v, o, do, lse, dq, dk, dv, causal, scale, workspace)
+    _check(load_library().attn_bwd(*args, _stream(stream)), "attn_bwd")
 
 
 def attn_decode_paged_workspace_size(num_seqs: int, Hq: int, Hkv: int, d: int, max_pages_per_seq: int,
@@ -306,6 +312,15 @@ def attn_debug_fwd_stall(q, k, v, o, lse, causal: bool, scale: float, stall_cta:
     st = lib.attn_debug_fwd_stall(*ptrs, *dims, float(scale), int(bool(causal)), int(stall_cta), int(stall_fill),
                                   int(timeout_ns), _stream(stream))
     _check(st, "attn_debug_fwd_stall")
+
+
+def attn_debug_bwd_stall(q, k, v, o, do, lse, dq, dk, dv, causal: bool, scale: float, stall_cta: int,
+                         stall_step: int, timeout_ns: int, workspace: torch.Tensor | None = None, stream=None) -> None:
+    """attn_bwd with the Q tile of one step left out in one CTA of the gradient kernel and
+    pipeline waits limited to timeout_ns (testing only)."""
+    args = _bwd_args(q, k, v, o, do, lse, dq, dk, dv, causal, scale, workspace)
+    st = load_library().attn_debug_bwd_stall(*args, int(stall_cta), int(stall_step), int(timeout_ns), _stream(stream))
+    _check(st, "attn_debug_bwd_stall")
 
 
 def attn_debug_decode_stall(q, k_pool, v_pool, block_table, seq_lens, page_size: int, o, lse, scale: float,

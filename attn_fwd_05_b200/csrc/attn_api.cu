@@ -438,9 +438,11 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Nq) {
   return ((size_t)B * Hq * Nq * sizeof(float) + 255) & ~(size_t)255;
 }
 
-attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-                     float* dq, float* dk, float* dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
-                     int causal, void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+
+attn_status bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                       float* dq, float* dk, float* dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                       int causal, void* workspace, size_t workspace_bytes, void* stream, const DebugStall* dbg) {
   if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.0f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
@@ -494,9 +496,20 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
   a.n_ktiles = (Nk + 127) / 128;
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.timeout_ns = kDefaultTimeoutNs;
+  a.timeout_ns = dbg != nullptr ? dbg->timeout_ns : kDefaultTimeoutNs;
+  a.dbg_stall_cta = dbg != nullptr ? dbg->cta : -1;
+  a.dbg_stall_step = dbg != nullptr ? dbg->fill : -1;
   float* delta = static_cast<float*>(workspace);
   return d == 64 ? launch_bwd<64>(a, o, dout, delta, st) : launch_bwd<128>(a, o, dout, delta, st);
+}
+
+}  // namespace
+
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                     float* dq, float* dk, float* dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                     int causal, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, workspace,
+                    workspace_bytes, stream, nullptr);
 }
 
 size_t attn_decode_paged_workspace_size(int num_seqs, int Hq, int Hkv, int d, int max_pages_per_seq,
@@ -642,6 +655,16 @@ attn_status attn_debug_fwd_stall(const void* q, const void* k, const void* v, vo
   if (stall_cta < 0 || stall_fill < 0 || timeout_ns == 0 || timeout_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;
   const DebugStall dbg{stall_cta, stall_fill, timeout_ns};
   return fwd_common(q, k, v, o, o_dtype, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, nullptr, stream, &dbg);
+}
+
+attn_status attn_debug_bwd_stall(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                 const float* lse, float* dq, float* dk, float* dv, int B, int Hq, int Hkv, int Nq,
+                                 int Nk, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                                 int stall_cta, int stall_step, uint64_t timeout_ns, void* stream) {
+  if (stall_cta < 0 || stall_step < 0 || timeout_ns == 0 || timeout_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;
+  const DebugStall dbg{stall_cta, stall_step, timeout_ns};
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, workspace,
+                    workspace_bytes, stream, &dbg);
 }
 
 attn_status attn_debug_decode_stall(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_table,

@@ -48,6 +48,10 @@ struct BwdArgs {
   int B, Hq, Hkv, Nq, Nk, group, causal, n_qtiles, n_ktiles;
   float scale, scale_log2;
   uint64_t timeout_ns;
+  // failure-path testing only (-1 in every normal call): CTA dbg_stall_cta leaves the Q
+  // tile of its step dbg_stall_step out, so the wait for it runs out after timeout_ns
+  int dbg_stall_cta;
+  int dbg_stall_step;
 };
 
 // The log-sum-exp in log2 units, with +inf for rows that must give P = 0 (outside the
@@ -274,6 +278,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
         for (; j < nsteps; ++j) {
           const int st = j & 1;
           if (j >= 2 && !mbar_wait(&bars->q_empty[st], ((j >> 1) - 1) & 1, abort_flag, a.timeout_ns)) break;
+          if (a.dbg_stall_cta == (int)blockIdx.x && j == a.dbg_stall_step) continue;  // left out (testing)
           mbar_arrive_expect_tx(&bars->q_full[st], C::TILE_BYTES);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c)
@@ -284,6 +289,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
         mbar_wait(&bars->fixed_full, 0, abort_flag, a.timeout_ns, false);
         for (int st = 0; st < 2 && st < j; ++st) {
           const int last = j - 1 - ((j - 1 - st) & 1);  // last step that used stage st
+          if (a.dbg_stall_cta == (int)blockIdx.x && last == a.dbg_stall_step) continue;
           mbar_wait(&bars->q_full[st], (last >> 1) & 1, abort_flag, a.timeout_ns, false);
         }
       }

@@ -321,6 +321,22 @@ attn_status attn_debug_fwd_stall(const void* q, const void* k, const void* v, vo
                                  int stall_fill, uint64_t timeout_ns, void* stream);
 
 /*
+ * attn_debug_bwd_stall — the same check for the backward pass: attn_bwd, with CTA
+ * `stall_cta` of the gradient kernel (one CTA per batch x KV head x 128-key tile)
+ * leaving out the Q tile of its step number `stall_step` (a step is one 128-query tile
+ * of one head of the group, in the order the CTA walks them) and pipeline waits limited
+ * to `timeout_ns` (1 ns .. 10 s).  dq, dk and dv are then undefined;
+ * attn_get_device_status reports ATTN_ERR_DEVICE_TIMEOUT.  A stall_step past the CTA's
+ * last step changes nothing.  For testing only.
+ */
+attn_status attn_debug_bwd_stall(const void* q, const void* k, const void* v, const void* o,
+                                 const void* dout, const float* lse, float* dq, float* dk,
+                                 float* dv, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                                 float scale, int causal, void* workspace,
+                                 size_t workspace_bytes, int stall_cta, int stall_step,
+                                 uint64_t timeout_ns, void* stream);
+
+/*
  * attn_debug_decode_stall — the same check for the paged decode: attn_decode_paged, with
  * CTA `stall_cta` of the split kernel leaving out its K/V piece number `stall_piece`
  * (16 tokens of K and V, in the order its producer gathers them) and pipeline waits

@@ -122,3 +122,75 @@ def test_stall_arguments_are_checked(cuda_device):
         with pytest.raises(ab.AttnError):
             ab.attn_debug_fwd_stall(q.to(dev), k.to(dev), v.to(dev), o, None, False, 0.1, cta, fill, lim)
     assert ab.attn_get_device_status() == 0
+
+
+def bwd_inputs(B, Hq, Hkv, N, d, causal, seed):
+    dev = torch.device("cuda:0")
+    shape = synth.PrefillShape(B=B, Hq=Hq, Hkv=Hkv, Nq=N, Nk=N, d=d, causal=causal)
+    q, k, v = (t.to(dev) for t in synth.prefill_inputs(shape, seed))
+    do = synth.upstream_grad(shape, seed).to(dev)
+    o = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    ab.attn_fwd(q, k, v, o, lse, causal, 1.0 / math.sqrt(d))
+    return q, k, v, o, do, lse
+
+
+def bwd_outputs(q, k):
+    return (torch.empty(q.shape, dtype=torch.float32, device=q.device),
+            torch.empty(k.shape, dtype=torch.float32, device=k.device),
+            torch.empty(k.shape, dtype=torch.float32, device=k.device))
+
+
+def same_gradients(a, b):
+    # dK and dV are summed in tensor memory in a fixed order: bit for bit; dQ is summed by
+    # additions in L2 in an order that varies: a few fp32 roundings apart
+    assert (a[0] - b[0]).abs().max().item() <= 1e-5 * b[0].abs().max().item()
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,causal,cta,step", [
+    (1, 4, 2, 512, 128, True, 0, 0),      # the first Q tile of CTA 0
+    (1, 4, 2, 512, 128, True, 3, 2),      # a later step of another CTA
+    (2, 8, 2, 2048, 64, True, 40, 5),     # d = 64, one CTA of 64 stalls
+])
+def test_backward_wait_runs_out_then_device_is_usable(B, Hq, Hkv, N, d, causal, cta, step, cuda_device):
+    assert ab.attn_get_device_status() == 0
+    q, k, v, o, do, lse = bwd_inputs(B, Hq, Hkv, N, d, causal, seed=500 + N + d)
+    scale = 1.0 / math.sqrt(d)
+    ref = bwd_outputs(q, k)
+    ab.attn_bwd(q, k, v, o, do, lse, *ref, causal, scale)
+    assert ab.attn_get_device_status() == 0
+    got = bwd_outputs(q, k)
+    t0 = time.perf_counter()
+    ab.attn_debug_bwd_stall(q, k, v, o, do, lse, *got, causal, scale, cta, step, LIMIT_NS)
+    status = ab.attn_get_device_status()
+    assert status == TIMEOUT, ab.attn_status_string(status)
+    assert time.perf_counter() - t0 < 5.0
+    assert ab.attn_get_device_status() == 0
+    # the same context, an ordinary call: the same gradients as before the stall
+    for t in got:
+        t.fill_(float("nan"))
+    ab.attn_bwd(q, k, v, o, do, lse, *got, causal, scale)
+    assert ab.attn_get_device_status() == 0
+    same_gradients(got, ref)
+
+
+def test_backward_stall_past_the_last_step_changes_nothing(cuda_device):
+    q, k, v, o, do, lse = bwd_inputs(1, 4, 2, 300, 128, True, seed=41)
+    scale = 1.0 / math.sqrt(128)
+    ref = bwd_outputs(q, k)
+    ab.attn_bwd(q, k, v, o, do, lse, *ref, True, scale)
+    got = bwd_outputs(q, k)
+    ab.attn_debug_bwd_stall(q, k, v, o, do, lse, *got, True, scale, 0, 1 << 30, LIMIT_NS)
+    assert ab.attn_get_device_status() == 0
+    same_gradients(got, ref)
+
+
+def test_backward_stall_rejects_bad_arguments(cuda_device):
+    q, k, v, o, do, lse = bwd_inputs(1, 2, 2, 128, 64, False, seed=42)
+    out = bwd_outputs(q, k)
+    for cta, step, limit in ((-1, 0, LIMIT_NS), (0, -1, LIMIT_NS), (0, 0, 0), (0, 0, 20_000_000_000)):
+        with pytest.raises(ab.AttnError) as e:
+            ab.attn_debug_bwd_stall(q, k, v, o, do, lse, *out, False, 0.125, cta, step, limit)
+        assert e.value.status == 1  # ATTN_ERR_INVALID_ARG
+    assert ab.attn_get_device_status() == 0
