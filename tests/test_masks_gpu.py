@@ -48,7 +48,7 @@ WINDOW_CASES = [
     (1, 4, 4, 333, 333, 128, 100),    # MHA q-tile pairs, ragged tail
     (2, 8, 2, 520, 520, 64, 300),     # window spanning block edges, d=64
     (1, 4, 2, 200, 600, 128, 130),    # Nq < Nk: bottom-right alignment
-    (1, 2, 1, 450, 450, 256, 200),    # d=256 (128-key blocks)
+    (1, 2, 1, 450, 450, 256, 200),    # d=256 (64-key blocks)
     (1, 2, 2, 300, 300, 256, 1),
     (1, 4, 2, 256, 256, 128, 10000),  # window wider than the sequence = causal
 ]

@@ -35,9 +35,9 @@ CASES = [
     (1, 2, 2, 512, 512, 256, False, 3.0),      # peaked d=256 (scores with std 9)
     (1, 2, 1, 300, 300, 256, True, 1.0),       # d=256 causal, ragged, GQA
     (1, 2, 2, 130, 70, 256, False, 1.0),       # d=256 Nk < one block
-    (1, 1, 1, 128, 128, 256, False, 1.0),      # d=256 exactly one 128-key visit
-    (1, 2, 1, 1000, 1000, 256, True, 1.0),     # d=256 up to 8 visits, the K/V ring wraps, ragged tail
-    (1, 2, 2, 200, 2300, 256, False, 2.0),     # d=256 18 visits of one q-tile, Nk ragged
+    (1, 1, 1, 128, 128, 256, False, 1.0),      # d=256 exactly one q-tile and one 128-key block
+    (1, 2, 1, 1000, 1000, 256, True, 1.0),     # d=256 causal, the K/V ring wraps several times, ragged tail
+    (1, 2, 2, 200, 2300, 256, False, 2.0),     # d=256 a long key row per q-tile, Nk ragged
 ]
 
 
