@@ -69,6 +69,8 @@ __device__ __forceinline__ bool stalled_fill(int stall_cta, int stall_fill, int 
 }
 
 constexpr int kMaskBlock = 128;  // block size of the block-sparse map
+constexpr int kUnitBand = 16;           // q-tile levels per band of the causal unit order
+constexpr int kUnitBandMinTiles = 64;   // q-tiles from which the levels are banded
 constexpr int kMaxVisits = 2048;  // blocks a CTA may visit under a block-sparse map
 
 struct TileJob {
@@ -402,8 +404,22 @@ __device__ __forceinline__ void unit_tiles(const FwdArgs& a, int u, int& b, int&
     const int hp_n = a.Hq / 2;
     int qt, rem;
     if (a.causal) {
-      qt = a.n_qtiles - 1 - u / (a.B * hp_n);
-      rem = u % (a.B * hp_n);
+      // Heaviest first: q-tile levels from the top.  Long sequences take the levels in
+      // bands of kUnitBand, and within a band the (batch, KV head) groups one after
+      // another, so that a round of CTAs streams the K/V of about two KV heads instead of
+      // all of them and their re-reads stay in L2 (16K causal GQA: DRAM reads 656 -> 508
+      // MB per launch, time unchanged within 1 %).  With fewer levels, one level a band.
+      const int per_level = a.B * hp_n;
+      const int L = a.n_qtiles >= kUnitBandMinTiles ? kUnitBand : 1;
+      const int band = u / (L * per_level);
+      const int in_band = u % (L * per_level);
+      const int lv_hi = a.n_qtiles - 1 - band * L;
+      const int nl = min(L, lv_hi + 1);  // the last band may be shorter
+      const int P = a.group / 2;         // head pairs of one KV head
+      const int gkv = in_band / (nl * P);
+      const int r2 = in_band % (nl * P);
+      qt = lv_hi - r2 / P;
+      rem = gkv * P + r2 % P;
     } else {
       qt = u % a.n_qtiles;
       rem = u / a.n_qtiles;

@@ -112,6 +112,7 @@ MULTI_UNIT = [
     (2, 16, 4, 4096, 64, True),    # 512: d = 64 (eight-stage ring)
     (1, 16, 2, 8192, 128, False),  # 512: non-causal order
     (3, 8, 2, 3000, 128, True),    # 288: ragged, the last q-tile of every head is partial
+    (2, 16, 4, 8300, 64, True),    # 1040: 65 q-tiles, levels taken in bands of 16, a short last band
 ]
 
 
