@@ -194,6 +194,8 @@ struct BwdCfg {
   static_assert(sizeof(BwdBars) <= 256, "barrier block");
 };
 
+constexpr int kBwdKeyBand = 64;  // key tiles per band of the grid order (long sequences)
+
 // Steps of a CTA: (query head of the group, q-tile), q-tiles from qt_lo on.
 __device__ __forceinline__ int kv_qt_lo(const BwdArgs& a, int kt) {
   if (!a.causal) return 0;
@@ -215,9 +217,18 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
   const int lane = threadIdx.x & 31;
 
   // causal: the first K/V tiles are seen by the most q-tiles, so they go first (longest
-  // processing time first); consecutive CTAs share a key-tile index
-  const int kt = blockIdx.x / (a.B * a.Hkv);
-  const int bkv = blockIdx.x % (a.B * a.Hkv);  // b * Hkv + kvh
+  // processing time first).  With 64 key tiles or more the key tiles are taken in bands of
+  // kBwdKeyBand, and within a band one (batch, KV head) after another: the CTAs in flight
+  // then belong to about two KV heads instead of all of them, and the Q, dO and dQ tiles
+  // they share stay in L2 (16K causal GQA: 22.2 -> 5.7 GB of DRAM traffic per call, the
+  // same time).  Fewer key tiles: one key tile a band, consecutive CTAs share it.
+  const int nbkv = a.B * a.Hkv;
+  const int KB = a.n_ktiles >= kBwdKeyBand ? kBwdKeyBand : 1;
+  const int kband = (int)blockIdx.x / (KB * nbkv);
+  const int in_band = (int)blockIdx.x % (KB * nbkv);
+  const int nk = min(KB, a.n_ktiles - kband * KB);  // the last band may be shorter
+  const int bkv = in_band / nk;                      // b * Hkv + kvh
+  const int kt = kband * KB + in_band % nk;
   const int b = bkv / a.Hkv, kvh = bkv % a.Hkv;
   const int k0 = kt * 128;
   const int qt_lo = kv_qt_lo(a, kt);
