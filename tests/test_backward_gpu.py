@@ -82,6 +82,7 @@ CASES = [
     (1, 2, 2, 1, 200, 64, False),       # one query row
     (1, 8, 2, 512, 512, 128, True),     # several tiles in both directions
     (1, 4, 2, 8200, 8200, 64, True),    # 65 key tiles: the grid takes them in bands of 64, a short last band
+    (1, 2, 1, 8200, 8200, 128, True),   # the same at d = 128 (dQ_step shares the dP^T columns)
 ]
 
 
